@@ -1,0 +1,144 @@
+"""Pins for the oracle's sparse attention and mask entry (CPU only).
+
+The independent reference is torch's fp64 scaled-dot-product attention on
+tensors the tests build themselves: dense attention over the dequantised
+INT8 Q/K (tau = -inf, all-ones mask), dense attention over K'/V' in which
+every skipped centroid group's rows are replaced by their mean (|g| equal
+keys contribute |g| * exp(q.kbar), which is exactly the ln|g| term), and a
+token-level boolean mask expanded from the logical block mask.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+import workloads
+
+
+def _head(name, b=0, h=0):
+    w = workloads.get(name)
+    q, k, v = workloads.head_qkv(w, b, h)
+    return w, q.float().numpy(), k.float().numpy(), v.float().numpy()
+
+
+def _dequant(x8, scale, rows):
+    out = np.zeros(x8.shape, np.float64)
+    for b, (r0, r1) in enumerate(oracle.block_rows(x8.shape[0], rows)):
+        out[r0:r1] = x8[r0:r1].astype(np.float64) * float(scale[b])
+    return out
+
+
+def _sdpa(q, k, v, scale, mask=None):
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64))[None, None]
+    m = None if mask is None else torch.from_numpy(mask)[None, None]
+    o = F.scaled_dot_product_attention(t(q), t(k), t(v), attn_mask=m, scale=scale)
+    return o[0, 0].numpy()
+
+
+@pytest.mark.parametrize("name", ["ragged_pe", "ragged_d64", "cross"])
+def test_all_kept_equals_dense_attention(name):
+    w, q, k, v = _head(name)
+    r = oracle.route_head(q, k, -math.inf)
+    assert r["keep"].all()
+    O, lse = oracle.sol_attention_head(r["q8"], r["q_scale"], r["k8"], r["k_scale"], v,
+                                       r["keep"], w.centroid_mode)
+    scale = 1.0 / math.sqrt(w.d)
+    ref = _sdpa(_dequant(r["q8"], r["q_scale"], 128), _dequant(r["k8"], r["k_scale"], 64), v, scale)
+    assert np.abs(O - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
+    # lse against a direct log-sum-exp of the dequantised logits
+    lg = scale * _dequant(r["q8"], r["q_scale"], 128) @ _dequant(r["k8"], r["k_scale"], 64).T
+    ref_lse = torch.logsumexp(torch.from_numpy(lg), dim=1).numpy()
+    assert np.abs(lse - ref_lse).max() <= 1e-10
+
+
+@pytest.mark.parametrize("name,mode", [("ragged_pe", 1), ("ragged_pe", 2),
+                                       ("ragged_d64", 2), ("cross", 1)])
+def test_centroids_equal_dense_attention_over_mean_replaced_kv(name, mode):
+    w, q, k, v = _head(name, 0, 1)
+    r = oracle.route_head(q, k, 0.7)
+    keep = r["keep"]
+    assert (~keep).any() and keep.any()
+    O, lse = oracle.sol_attention_head(r["q8"], r["q_scale"], r["k8"], r["k_scale"], v, keep, mode)
+    Qd = _dequant(r["q8"], r["q_scale"], 128)
+    Kd = _dequant(r["k8"], r["k_scale"], 64)
+    Vd = np.asarray(v, np.float64)
+    scale = 1.0 / math.sqrt(w.d)
+    Lq, Lk = Qd.shape[0], Kd.shape[0]
+    for i, (r0, r1) in enumerate(oracle.block_rows(Lq, 128)):
+        K2, V2 = Kd.copy(), Vd.copy()
+        for j, (t0, t1) in enumerate(oracle.block_rows(Lk, 64)):
+            if keep[i, j]:
+                continue
+            spans = [(t0, t1)] if mode == 1 else [(t0, min(t1, t0 + 32)), (min(t1, t0 + 32), t1)]
+            for g0, g1 in spans:
+                if g1 > g0:
+                    K2[g0:g1] = Kd[g0:g1].mean(axis=0)
+                    V2[g0:g1] = Vd[g0:g1].mean(axis=0)
+        ref = _sdpa(Qd[r0:r1], K2, V2, scale)
+        assert np.abs(O[r0:r1] - ref).max() <= 1e-10, (i, np.abs(O[r0:r1] - ref).max())
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_identical_token_block_same_kept_or_skipped(mode):
+    w, q, k, v = _head("ragged_pe")
+    k = k.copy(); v = v.copy()
+    k[320:384] = k[320]                 # key block 5: 64 identical tokens
+    v[320:384] = v[320]
+    r = oracle.route_head(q, k, 1.0)
+    keep = r["keep"].copy()
+    keep[:, 5] = True
+    O1, l1 = oracle.sol_attention_head(r["q8"], r["q_scale"], r["k8"], r["k_scale"], v, keep, mode)
+    keep[:, 5] = False
+    O2, l2 = oracle.sol_attention_head(r["q8"], r["q_scale"], r["k8"], r["k_scale"], v, keep, mode)
+    assert np.abs(O1 - O2).max() <= 1e-12
+    assert np.abs(l1 - l2).max() <= 1e-12
+
+
+def test_mask_entry_matches_token_level_masked_dense():
+    w, q, k, v = _head("lcsa_small")
+    r = oracle.route_head(q, k, -math.inf)
+    logical = workloads.block_mask(w)[0, 0].numpy()
+    allowed = oracle.physical_allowed(logical, w.nKB)
+    O, lse = oracle.masked_attention_head(r["q8"], r["q_scale"], r["k8"], r["k_scale"], v, allowed)
+    Lq, Lk = w.Lq, w.Lk
+    tok = np.zeros((Lq, Lk), bool)
+    for i in range(logical.shape[0]):
+        for x in range(logical.shape[1]):
+            if logical[i, x]:
+                tok[128 * i:128 * i + 128, 128 * x:128 * x + 128] = True
+    ref = _sdpa(_dequant(r["q8"], r["q_scale"], 128), _dequant(r["k8"], r["k_scale"], 64), v,
+                1.0 / math.sqrt(w.d), tok)
+    assert np.abs(O - ref).max() <= 1e-12
+
+
+def test_mask_all_ones_is_dense_and_empty_row_is_zero():
+    w, q, k, v = _head("cross")
+    r = oracle.route_head(q, k, -math.inf)
+    nQB, nLK = w.nQB, w.nLK
+    ones = np.ones((nQB, nLK), np.uint8)
+    ones[2] = 0                                    # query block 2 sees nothing
+    allowed = oracle.physical_allowed(ones, w.nKB)
+    O, lse = oracle.masked_attention_head(r["q8"], r["q_scale"], r["k8"], r["k_scale"], v, allowed)
+    Od, _ = oracle.sol_attention_head(r["q8"], r["q_scale"], r["k8"], r["k_scale"], v,
+                                      np.ones((nQB, w.nKB), bool), 0)
+    rows = np.r_[0:256, 384:w.Lq]
+    assert np.abs(O[rows] - Od[rows]).max() == 0
+    assert (O[256:384] == 0).all() and np.isneginf(lse[256:384]).all()
+
+
+def test_physical_allowed_maps_logical_pairs():
+    logical = np.array([[1, 0, 1], [0, 1, 0]], np.uint8)
+    phys = oracle.physical_allowed(logical, 5)     # 5 physical = ceil(300/64) for Lk = 300
+    assert phys.astype(int).tolist() == [[1, 1, 0, 0, 1], [0, 0, 1, 1, 0]]
+
+
+def test_softmax_scale_argument():
+    w, q, k, v = _head("cross")
+    r = oracle.route_head(q, k, -math.inf)
+    O, _ = oracle.sol_attention_head(r["q8"], r["q_scale"], r["k8"], r["k_scale"], v, r["keep"], 1,
+                                     softmax_scale=0.05)
+    ref = _sdpa(_dequant(r["q8"], r["q_scale"], 128), _dequant(r["k8"], r["k_scale"], 64), v, 0.05)
+    assert np.abs(O - ref).max() <= 1e-12

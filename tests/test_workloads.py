@@ -1,0 +1,54 @@
+"""Checks of the seeded input generator (CPU only)."""
+import numpy as np
+import torch
+
+import workloads
+
+
+def test_lcsa_mask_density_is_21_over_64():
+    w = workloads.get("lcsa")
+    m = workloads.block_mask(w)
+    assert tuple(m.shape) == (1, 1, 96, 96)
+    assert int(m.sum()) * 64 == 21 * 96 * 96
+
+
+def test_lcsa_window_rule():
+    m = workloads.lcsa_block_mask(128 * 30, 128 * 30, 384, 2)   # 3 blocks per frame
+    for i in range(30):
+        fq = i // 3
+        for x in range(30):
+            fk = x // 3
+            assert bool(m[i, x]) == (fq - 2 <= fk <= fq)
+
+
+def test_heads_reproducible_and_independent():
+    w = workloads.get("ragged_pe")
+    a = workloads.head_qkv(w, 1, 2)
+    b = workloads.head_qkv(w, 1, 2)
+    c = workloads.head_qkv(w, 0, 2)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+    assert not torch.equal(a[0], c[0])
+    Q, K, V = workloads.batch_qkv(w)
+    assert torch.equal(Q[1, 2], a[0]) and torch.equal(V[1, 2], a[2])
+    assert Q.dtype == torch.bfloat16 and tuple(Q.shape) == (2, 3, 1000, 128)
+
+
+def test_config_shapes():
+    assert workloads.get("wan14b").Lq == 32760
+    assert workloads.get("h3").Lq == 85696
+    assert workloads.get("h3").nQB == 670 and workloads.get("h3").nKB == 1339
+    assert workloads.get("wan13b").nKB == 512
+
+
+def test_pe_signal_and_prefix():
+    w = workloads.get("prefix_small")
+    q, k, v = workloads.head_qkv(w, 0, 0)
+    qf = q.float().numpy()
+    pre, vid = qf[:256], qf[256:]
+    assert abs(pre.std() - 1.0) < 0.05             # prefix: plain N(0,1)
+    assert vid.std() > 1.4                         # video: signal + noise (var ~ 3)
+    # Q and K share the signal, so their video rows correlate strongly
+    kf = k.float().numpy()[256:]
+    corr = np.corrcoef(vid.ravel(), kf.ravel())[0, 1]
+    assert corr > 0.5
