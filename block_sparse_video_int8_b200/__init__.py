@@ -1,0 +1,276 @@
+"""Python binding of ``libbsva.so``, the block-sparse INT8 video attention library.
+
+Argument marshalling only: every step of the method runs in the CUDA kernels
+behind the C ABI declared in ``include/bsva.h``. PyTorch supplies device
+memory and the current stream. There is no CPU or fallback path: if the
+library is missing or was built for another ABI, ``load()`` raises.
+
+Entry points (same names as the C ABI):
+
+* ``quantize_qk(q, k)``                      per-block INT8 Q/K, scales, pools
+* ``sparse_attn_route(q, k, tau, n_prefix)`` quantise + proxy score + Sol rule
+* ``sparse_attn_fwd(route, v, mode)``        kept blocks exact + centroids
+* ``masked_block_attn_fwd(q8, ..., mask)``   explicit logical 128x128 block mask
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+__all__ = [
+    "BsvaError", "load", "lib_path", "Route", "Shape", "abi_version",
+    "workspace_bytes", "quantize_qk", "sparse_attn_route", "sparse_attn_fwd",
+    "masked_block_attn_fwd", "check_status", "selftest_timeout", "new_workspace",
+]
+
+ABI_VERSION = 1
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB = None
+
+STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA",
+          5: "DEVICE_TIMEOUT"}
+
+
+class BsvaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"bsva error {code} ({STATUS.get(code, '?')}): {msg}")
+        self.code = code
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("Lq", ctypes.c_int),
+                ("Lk", ctypes.c_int), ("d", ctypes.c_int), ("n_prefix", ctypes.c_int)]
+
+
+def lib_path() -> str:
+    return os.path.join(_HERE, "libbsva.so")
+
+
+_P = ctypes.c_void_p
+_SIGS = {
+    "bsva_abi_version": (ctypes.c_int, []),
+    "bsva_last_error": (ctypes.c_char_p, []),
+    "bsva_workspace_bytes": (ctypes.c_size_t, [Shape, ctypes.c_int]),
+    "bsva_quantize_qk": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "sparse_attn_route": (ctypes.c_int, [Shape, _P, _P, ctypes.c_double, _P, _P, _P, _P, _P, _P,
+                                         _P, _P, _P, _P, _P]),
+    "sparse_attn_fwd": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int,
+                                       ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]),
+    "masked_block_attn_fwd": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, _P, ctypes.c_int,
+                                             ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]),
+    "bsva_check_status": (ctypes.c_int, [_P, _P]),
+    "bsva_selftest_timeout": (ctypes.c_int, [_P, ctypes.c_size_t, ctypes.c_longlong, _P]),
+}
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load the CUDA library (once) and check its ABI version; raise if unavailable."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = path or lib_path()
+    if not os.path.exists(path):
+        raise FileNotFoundError(
+            f"libbsva.so not found at {path}; build it with "
+            "`python -m block_sparse_video_int8_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    ver = lib.bsva_abi_version()
+    if ver != ABI_VERSION:
+        raise RuntimeError(f"{path} has ABI version {ver}, this binding expects {ABI_VERSION}")
+    _LIB = lib
+    return lib
+
+
+def abi_version() -> int:
+    return load().bsva_abi_version()
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise BsvaError(rc, load().bsva_last_error().decode(errors="replace"))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, dtype, shape, name):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _shape_of(q, k, n_prefix=0) -> Shape:
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q and k must be [B, H, L, d]")
+    B, H, Lq, d = q.shape
+    if tuple(k.shape[:2]) != (B, H) or k.shape[3] != d:
+        raise ValueError(f"k shape {tuple(k.shape)} does not match q {tuple(q.shape)}")
+    return Shape(B, H, Lq, k.shape[2], d, n_prefix)
+
+
+def workspace_bytes(shape: Shape, centroid_mode: int) -> int:
+    n = load().bsva_workspace_bytes(shape, centroid_mode)
+    if n == 0:
+        raise BsvaError(1, f"bad shape or centroid_mode for a workspace: {_fmt(shape)}, mode {centroid_mode}")
+    return n
+
+
+def _fmt(s: Shape) -> str:
+    return f"B={s.B} H={s.H} Lq={s.Lq} Lk={s.Lk} d={s.d} n_prefix={s.n_prefix}"
+
+
+def new_workspace(shape: Shape, centroid_mode: int, device=None) -> torch.Tensor:
+    """A zeroed device workspace (uint8) large enough for ``shape`` and mode."""
+    n = workspace_bytes(shape, centroid_mode)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+@dataclass
+class Route:
+    """Outputs of the routing step (all device tensors)."""
+    shape: Shape
+    tau: float
+    q8: torch.Tensor
+    q_scale: torch.Tensor
+    k8: torch.Tensor
+    k_scale: torch.Tensor
+    q_pool: torch.Tensor
+    k_pool: torch.Tensor
+    kept_mask: torch.Tensor
+    kept_idx: torch.Tensor
+    kept_cnt: torch.Tensor
+    row_stats: torch.Tensor | None
+
+
+def _alloc_quant(s: Shape, dev):
+    nQB, nKB = -(-s.Lq // 128), -(-s.Lk // 64)
+    return dict(
+        q8=torch.empty((s.B, s.H, s.Lq, s.d), dtype=torch.int8, device=dev),
+        q_scale=torch.empty((s.B, s.H, nQB), dtype=torch.float32, device=dev),
+        k8=torch.empty((s.B, s.H, s.Lk, s.d), dtype=torch.int8, device=dev),
+        k_scale=torch.empty((s.B, s.H, nKB), dtype=torch.float32, device=dev),
+        q_pool=torch.empty((s.B, s.H, nQB, s.d), dtype=torch.int32, device=dev),
+        k_pool=torch.empty((s.B, s.H, nKB, 2, s.d), dtype=torch.int32, device=dev),
+    )
+
+
+def quantize_qk(q: torch.Tensor, k: torch.Tensor, out: dict | None = None, stream=None) -> dict:
+    """Per-block INT8 Q/K with scales and sum-pools (C ABI ``bsva_quantize_qk``)."""
+    lib = load()
+    s = _shape_of(q, k)
+    _need(q, torch.bfloat16, None, "q")
+    _need(k, torch.bfloat16, None, "k")
+    o = out or _alloc_quant(s, q.device)
+    _check(lib.bsva_quantize_qk(s, _ptr(q), _ptr(k), _ptr(o["q8"]), _ptr(o["q_scale"]), _ptr(o["k8"]),
+                                _ptr(o["k_scale"]), _ptr(o["q_pool"]), _ptr(o["k_pool"]),
+                                _stream(stream)))
+    return o
+
+
+def sparse_attn_route(q: torch.Tensor, k: torch.Tensor, tau: float, n_prefix: int = 0,
+                      row_stats: bool = False, out: Route | None = None, stream=None) -> Route:
+    """Quantise, score and route (C ABI ``sparse_attn_route``)."""
+    lib = load()
+    s = _shape_of(q, k, n_prefix)
+    _need(q, torch.bfloat16, None, "q")
+    _need(k, torch.bfloat16, None, "k")
+    nQB, nKB = -(-s.Lq // 128), -(-s.Lk // 64)
+    if out is None:
+        dev = q.device
+        o = _alloc_quant(s, dev)
+        out = Route(shape=s, tau=tau, **o,
+                    kept_mask=torch.empty((s.B, s.H, nQB, nKB), dtype=torch.uint8, device=dev),
+                    kept_idx=torch.empty((s.B, s.H, nQB, nKB), dtype=torch.int32, device=dev),
+                    kept_cnt=torch.empty((s.B, s.H, nQB), dtype=torch.int32, device=dev),
+                    row_stats=(torch.empty((s.B, s.H, nQB, 3), dtype=torch.float64, device=dev)
+                               if row_stats else None))
+    else:
+        out.shape, out.tau = s, tau
+    _check(lib.sparse_attn_route(s, _ptr(q), _ptr(k), ctypes.c_double(tau), _ptr(out.q8),
+                                 _ptr(out.q_scale), _ptr(out.k8), _ptr(out.k_scale), _ptr(out.q_pool),
+                                 _ptr(out.k_pool), _ptr(out.kept_mask), _ptr(out.kept_idx),
+                                 _ptr(out.kept_cnt), _ptr(out.row_stats), _stream(stream)))
+    return out
+
+
+def sparse_attn_fwd(route: Route, v: torch.Tensor, centroid_mode: int, softmax_scale: float = 0.0,
+                    with_lse: bool = False, workspace: torch.Tensor | None = None,
+                    out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                    stream=None):
+    """Sparse attention over the routed blocks plus centroids (C ABI ``sparse_attn_fwd``).
+
+    Returns ``out`` (bf16 [B, H, Lq, d]) or ``(out, lse)`` when ``with_lse``.
+    """
+    lib = load()
+    s = route.shape
+    _need(v, torch.bfloat16, (s.B, s.H, s.Lk, s.d), "v")
+    if workspace is None:
+        workspace = new_workspace(s, centroid_mode, v.device)
+    if out is None:
+        out = torch.empty((s.B, s.H, s.Lq, s.d), dtype=torch.bfloat16, device=v.device)
+    if with_lse and lse is None:
+        lse = torch.empty((s.B, s.H, s.Lq), dtype=torch.float32, device=v.device)
+    _check(lib.sparse_attn_fwd(s, _ptr(route.q8), _ptr(route.q_scale), _ptr(route.k8),
+                               _ptr(route.k_scale), _ptr(route.k_pool), _ptr(v), _ptr(route.kept_mask),
+                               _ptr(route.kept_idx), _ptr(route.kept_cnt), centroid_mode,
+                               ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace),
+                               workspace.numel(), _stream(stream)))
+    return (out, lse) if with_lse else out
+
+
+def masked_block_attn_fwd(q8, q_scale, k8, k_scale, v, block_mask, softmax_scale: float = 0.0,
+                          with_lse: bool = False, workspace=None, out=None, lse=None, stream=None):
+    """Attention over an explicit logical 128x128 block mask (C ABI ``masked_block_attn_fwd``)."""
+    lib = load()
+    B, H, Lq, d = q8.shape
+    Lk = k8.shape[2]
+    s = Shape(B, H, Lq, Lk, d, 0)
+    _need(q8, torch.int8, None, "q8")
+    _need(k8, torch.int8, (B, H, Lk, d), "k8")
+    _need(v, torch.bfloat16, (B, H, Lk, d), "v")
+    _need(block_mask, torch.uint8, None, "block_mask")
+    if block_mask.dim() != 4 or block_mask.shape[0] != B or block_mask.shape[2:] != (-(-Lq // 128), -(-Lk // 128)):
+        raise ValueError(f"block_mask shape {tuple(block_mask.shape)} is not [B, Hm, nQB, nLK]")
+    mask_heads = block_mask.shape[1]
+    if workspace is None:
+        workspace = new_workspace(s, 0, v.device)
+    if out is None:
+        out = torch.empty((B, H, Lq, d), dtype=torch.bfloat16, device=v.device)
+    if with_lse and lse is None:
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=v.device)
+    _check(lib.masked_block_attn_fwd(s, _ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(k_scale), _ptr(v),
+                                     _ptr(block_mask), mask_heads, ctypes.c_float(softmax_scale),
+                                     _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+                                     _stream(stream)))
+    return (out, lse) if with_lse else out
+
+
+def check_status(workspace: torch.Tensor, stream=None):
+    """Synchronise and raise BsvaError if a device-side wait timed out."""
+    _check(load().bsva_check_status(_ptr(workspace), _stream(stream)))
+
+
+def selftest_timeout(workspace: torch.Tensor, limit_ns: int, stream=None):
+    """Launch the bounded-wait self test (a wait that is meant to run out)."""
+    _check(load().bsva_selftest_timeout(_ptr(workspace), workspace.numel(), int(limit_ns),
+                                        _stream(stream)))

@@ -1,0 +1,307 @@
+// api.cu -- the C ABI (include/bsva.h): argument validation, TMA descriptor
+// encoding, workspace carving and kernel launches on the caller's stream.
+// No entry point allocates, frees or synchronises device memory (except
+// bsva_check_status, whose job is to synchronise), and none falls back to
+// another path: a bad argument or an unsupported device returns an error code
+// and leaves every output untouched.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+
+namespace bsva {
+bool route_supported(int nKB, int d);
+}
+
+using namespace bsva;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int ok() {
+  g_last_error.clear();
+  return BSVA_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(BSVA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per device-side wait
+
+// ------------------------------------------------------------- device check
+int check_device() {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int major = 0, minor = 0;
+  e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0)
+    return fail(BSVA_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a (B200) only", dev,
+                major, minor);
+  return BSVA_OK;
+}
+
+// ------------------------------------------------------------ validation
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_shape(const bsva_shape& s) {
+  if (s.B < 1 || s.H < 1 || s.Lq < 1 || s.Lk < 1)
+    return fail(BSVA_ERR_INVALID_ARG, "shape: B, H, Lq, Lk must be >= 1 (got %d, %d, %d, %d)", s.B, s.H, s.Lq, s.Lk);
+  if (s.d != 64 && s.d != 128) return fail(BSVA_ERR_UNSUPPORTED, "head dim d = %d; supported: 64, 128", s.d);
+  if (s.n_prefix < 0 || s.n_prefix % 128 != 0)
+    return fail(BSVA_ERR_INVALID_ARG, "n_prefix = %d must be a non-negative multiple of 128", s.n_prefix);
+  if (s.Lq > (1 << 30) || s.Lk > (1 << 30)) return fail(BSVA_ERR_INVALID_ARG, "sequence length too large");
+  if (size_t(s.B) * s.H > 65535u) return fail(BSVA_ERR_INVALID_ARG, "B*H must be <= 65535");
+  const size_t nQB = (size_t(s.Lq) + 127) / 128;
+  if (size_t(s.B) * s.H * nQB > 0x7fffffffu) return fail(BSVA_ERR_INVALID_ARG, "too many query blocks");
+  return BSVA_OK;
+}
+
+#define REQUIRE_PTR(p, align)                                                                          \
+  do {                                                                                                 \
+    if ((p) == nullptr) return fail(BSVA_ERR_INVALID_ARG, "%s is NULL", #p);                           \
+    if (!aligned((p), (align))) return fail(BSVA_ERR_INVALID_ARG, "%s is not %d-byte aligned", #p, (align)); \
+  } while (0)
+
+// ----------------------------------------------------------- tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+int get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) return fail(BSVA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+  return BSVA_OK;
+}
+
+// 3-D map over [heads][rows][inner] with a box of [1][box_rows][box_inner].
+int encode_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t inner,
+               uint64_t rows, uint64_t heads, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw,
+               const char* what) {
+  cuuint64_t dims[3] = {inner, rows, heads};
+  cuuint64_t strides[2] = {inner * elem_bytes, rows * inner * elem_bytes};
+  cuuint32_t box[3] = {box_inner, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(BSVA_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed with %d", what, int(r));
+  return BSVA_OK;
+}
+
+int check_workspace(void* ws, size_t bytes, size_t need) {
+  if (ws == nullptr) return fail(BSVA_ERR_WORKSPACE, "workspace is NULL (need %zu bytes)", need);
+  if (!aligned(ws, 256)) return fail(BSVA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (bytes < need) return fail(BSVA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", bytes, need);
+  return BSVA_OK;
+}
+
+// Shared tail of both attention entry points.
+int run_attention(const bsva_shape& s, const int8_t* q8, const float* q_scale, const int8_t* k8,
+                  const float* k_scale, const void* v, const uint8_t* kept_mask, const int32_t* kept_idx,
+                  const int32_t* kept_cnt, int centroid_mode, float softmax_scale, void* out, float* lse,
+                  unsigned char* ws, const WsLayout& L, cudaStream_t st) {
+  int rc = get_encoder();
+  if (rc) return rc;
+  const uint64_t BH = uint64_t(s.B) * s.H;
+  AttnMaps maps;
+  const CUtensorMapSwizzle swq = s.d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if ((rc = encode_map(&maps.q8, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.d, s.Lq, BH, s.d, QB, swq, "q8"))) return rc;
+  if ((rc = encode_map(&maps.k8, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.d, s.Lk, BH, s.d, KB, swq, "k8"))) return rc;
+  if ((rc = encode_map(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, s.d, s.Lk, BH, 64, KB,
+                       CU_TENSOR_MAP_SWIZZLE_128B, "v")))
+    return rc;
+  if (centroid_mode > 0) {
+    const uint64_t nCR = uint64_t(L.nCT) * 64;
+    if ((rc = encode_map(&maps.ck8, ws + L.ck8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.d, nCR, BH, s.d, KB, swq, "ck8")))
+      return rc;
+    if ((rc = encode_map(&maps.cv, ws + L.cv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, s.d, nCR, BH, 64, KB,
+                         CU_TENSOR_MAP_SWIZZLE_128B, "cv")))
+      return rc;
+  } else {
+    maps.ck8 = maps.k8;
+    maps.cv = maps.v;
+  }
+  AttnArgs a{};
+  a.B = s.B; a.H = s.H; a.Lq = s.Lq; a.Lk = s.Lk; a.d = s.d; a.n_prefix = s.n_prefix;
+  a.nQB = (s.Lq + QB - 1) / QB;
+  a.nKB = (s.Lk + KB - 1) / KB;
+  a.centroid_mode = centroid_mode;
+  a.nCT = L.nCT;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf(float(s.d));
+  a.scale_log2e = scale * 1.4426950408889634f;
+  a.q_scale = q_scale;
+  a.k_scale = k_scale;
+  a.kept_idx = kept_idx;
+  a.kept_cnt = kept_cnt;
+  a.kept_mask = kept_mask;
+  a.cfac = centroid_mode > 0 ? reinterpret_cast<const float*>(ws + L.cfac) : nullptr;
+  a.cbias = centroid_mode > 0 ? reinterpret_cast<const float*>(ws + L.cbias) : nullptr;
+  a.order = nullptr;
+  a.out = reinterpret_cast<__nv_bfloat16*>(out);
+  a.lse = lse;
+  a.status = reinterpret_cast<uint32_t*>(ws + L.status);
+  a.wait_limit_ns = kWaitLimitNs;
+  cudaError_t e = launch_attention(a, maps, st);
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+int bsva_abi_version(void) { return BSVA_ABI_VERSION; }
+
+const char* bsva_last_error(void) { return g_last_error.c_str(); }
+
+size_t bsva_workspace_bytes(bsva_shape s, int centroid_mode) {
+  if (check_shape(s) != BSVA_OK || centroid_mode < 0 || centroid_mode > 2) return 0;
+  return ws_layout(s, centroid_mode).total;
+}
+
+int bsva_quantize_qk(bsva_shape s, const void* q, const void* k, int8_t* q8, float* q_scale, int8_t* k8,
+                     float* k_scale, int32_t* q_pool, int32_t* k_pool, bsva_stream_t stream) {
+  int rc;
+  if ((rc = check_shape(s))) return rc;
+  REQUIRE_PTR(q, 16); REQUIRE_PTR(k, 16); REQUIRE_PTR(q8, 16); REQUIRE_PTR(k8, 16);
+  REQUIRE_PTR(q_scale, 4); REQUIRE_PTR(k_scale, 4); REQUIRE_PTR(q_pool, 16); REQUIRE_PTR(k_pool, 16);
+  if ((rc = check_device())) return rc;
+  cudaError_t e = launch_quant_pool(s, reinterpret_cast<const __nv_bfloat16*>(q),
+                                    reinterpret_cast<const __nv_bfloat16*>(k), q8, q_scale, k8, k_scale, q_pool,
+                                    k_pool, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "quant_pool launch");
+  return ok();
+}
+
+int sparse_attn_route(bsva_shape s, const void* q, const void* k, double tau, int8_t* q8, float* q_scale, int8_t* k8,
+                      float* k_scale, int32_t* q_pool, int32_t* k_pool, uint8_t* kept_mask, int32_t* kept_idx,
+                      int32_t* kept_cnt, double* row_stats, bsva_stream_t stream) {
+  int rc;
+  if ((rc = check_shape(s))) return rc;
+  if (std::isnan(tau)) return fail(BSVA_ERR_INVALID_ARG, "tau is NaN");
+  if (std::isinf(tau) && tau > 0) return fail(BSVA_ERR_INVALID_ARG, "tau = +inf is not a routing threshold");
+  REQUIRE_PTR(q, 16); REQUIRE_PTR(k, 16); REQUIRE_PTR(q8, 16); REQUIRE_PTR(k8, 16);
+  REQUIRE_PTR(q_scale, 4); REQUIRE_PTR(k_scale, 4); REQUIRE_PTR(q_pool, 16); REQUIRE_PTR(k_pool, 16);
+  REQUIRE_PTR(kept_mask, 1); REQUIRE_PTR(kept_idx, 4); REQUIRE_PTR(kept_cnt, 4);
+  if (row_stats && !aligned(row_stats, 8)) return fail(BSVA_ERR_INVALID_ARG, "row_stats is not 8-byte aligned");
+  const int nKB = (s.Lk + KB - 1) / KB;
+  if (!route_supported(nKB, s.d))
+    return fail(BSVA_ERR_UNSUPPORTED, "Lk = %d: a routing row does not fit shared memory", s.Lk);
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_quant_pool(s, reinterpret_cast<const __nv_bfloat16*>(q),
+                                    reinterpret_cast<const __nv_bfloat16*>(k), q8, q_scale, k8, k_scale, q_pool,
+                                    k_pool, st);
+  if (e != cudaSuccess) return cuda_fail(e, "quant_pool launch");
+  e = launch_route(s, tau, q_pool, k_pool, k_scale, kept_mask, kept_idx, kept_cnt, row_stats, st);
+  if (e != cudaSuccess) return cuda_fail(e, "route launch");
+  return ok();
+}
+
+int sparse_attn_fwd(bsva_shape s, const int8_t* q8, const float* q_scale, const int8_t* k8, const float* k_scale,
+                    const int32_t* k_pool, const void* v, const uint8_t* kept_mask, const int32_t* kept_idx,
+                    const int32_t* kept_cnt, int centroid_mode, float softmax_scale, void* out, float* lse,
+                    void* workspace, size_t workspace_bytes, bsva_stream_t stream) {
+  int rc;
+  if ((rc = check_shape(s))) return rc;
+  if (centroid_mode != 1 && centroid_mode != 2)
+    return fail(BSVA_ERR_INVALID_ARG, "centroid_mode = %d; use 1 (1x64) or 2 (2x32)", centroid_mode);
+  if (std::isnan(softmax_scale) || std::isinf(softmax_scale))
+    return fail(BSVA_ERR_INVALID_ARG, "softmax_scale must be finite");
+  REQUIRE_PTR(q8, 16); REQUIRE_PTR(q_scale, 4); REQUIRE_PTR(k8, 16); REQUIRE_PTR(k_scale, 4);
+  REQUIRE_PTR(k_pool, 16); REQUIRE_PTR(v, 16); REQUIRE_PTR(kept_mask, 1); REQUIRE_PTR(kept_idx, 4);
+  REQUIRE_PTR(kept_cnt, 4); REQUIRE_PTR(out, 16);
+  if (lse && !aligned(lse, 4)) return fail(BSVA_ERR_INVALID_ARG, "lse is not 4-byte aligned");
+  const WsLayout L = ws_layout(s, centroid_mode);
+  if ((rc = check_workspace(workspace, workspace_bytes, L.total))) return rc;
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  cudaError_t e = launch_centroids(s, centroid_mode, L.nCT, k_pool, k_scale, reinterpret_cast<const __nv_bfloat16*>(v),
+                                   reinterpret_cast<int8_t*>(ws + L.ck8), reinterpret_cast<__nv_bfloat16*>(ws + L.cv),
+                                   reinterpret_cast<float*>(ws + L.cfac), reinterpret_cast<float*>(ws + L.cbias), st);
+  if (e != cudaSuccess) return cuda_fail(e, "centroid launch");
+  return run_attention(s, q8, q_scale, k8, k_scale, v, kept_mask, kept_idx, kept_cnt, centroid_mode, softmax_scale,
+                       out, lse, ws, L, st);
+}
+
+int masked_block_attn_fwd(bsva_shape s, const int8_t* q8, const float* q_scale, const int8_t* k8,
+                          const float* k_scale, const void* v, const uint8_t* block_mask, int mask_heads,
+                          float softmax_scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                          bsva_stream_t stream) {
+  int rc;
+  if ((rc = check_shape(s))) return rc;
+  if (mask_heads != 1 && mask_heads != s.H)
+    return fail(BSVA_ERR_INVALID_ARG, "mask_heads = %d must be 1 or H = %d", mask_heads, s.H);
+  if (std::isnan(softmax_scale) || std::isinf(softmax_scale))
+    return fail(BSVA_ERR_INVALID_ARG, "softmax_scale must be finite");
+  REQUIRE_PTR(q8, 16); REQUIRE_PTR(q_scale, 4); REQUIRE_PTR(k8, 16); REQUIRE_PTR(k_scale, 4);
+  REQUIRE_PTR(v, 16); REQUIRE_PTR(block_mask, 1); REQUIRE_PTR(out, 16);
+  if (lse && !aligned(lse, 4)) return fail(BSVA_ERR_INVALID_ARG, "lse is not 4-byte aligned");
+  const WsLayout L = ws_layout(s, 0);
+  if ((rc = check_workspace(workspace, workspace_bytes, L.total))) return rc;
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  int32_t* kidx = reinterpret_cast<int32_t*>(ws + L.kidx);
+  int32_t* kcnt = reinterpret_cast<int32_t*>(ws + L.kcnt);
+  cudaError_t e = launch_mask_expand(s, block_mask, mask_heads, kidx, kcnt, st);
+  if (e != cudaSuccess) return cuda_fail(e, "mask expansion launch");
+  return run_attention(s, q8, q_scale, k8, k_scale, v, nullptr, kidx, kcnt, 0, softmax_scale, out, lse, ws, L, st);
+}
+
+int bsva_check_status(void* workspace, bsva_stream_t stream) {
+  if (workspace == nullptr) return fail(BSVA_ERR_WORKSPACE, "workspace is NULL");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
+  if (word != 0) {
+    e = cudaMemsetAsync(workspace, 0, sizeof(word), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
+  }
+  if (word & kStatusTimeout)
+    return fail(BSVA_ERR_DEVICE_TIMEOUT, "a device-side wait ran out of time; outputs of that call are invalid");
+  return ok();
+}
+
+int bsva_selftest_timeout(void* workspace, size_t workspace_bytes, long long limit_ns, bsva_stream_t stream) {
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < 256)
+    return fail(BSVA_ERR_WORKSPACE, "workspace must be non-NULL, 256-byte aligned, >= 256 bytes");
+  if (limit_ns < 1000 || limit_ns > 1000000000LL)
+    return fail(BSVA_ERR_INVALID_ARG, "limit_ns = %lld outside [1e3, 1e9]", limit_ns);
+  int rc;
+  if ((rc = check_device())) return rc;
+  cudaError_t e = launch_selftest_timeout(static_cast<uint32_t*>(workspace), uint64_t(limit_ns),
+                                          reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
+  return ok();
+}
+
+}  // extern "C"

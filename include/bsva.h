@@ -1,0 +1,168 @@
+/*
+ * bsva.h -- C ABI of the block-sparse INT8 video attention library (sm_100a).
+ *
+ * The method: every 128-token query block scores each 64-token key block with
+ * a cheap proxy on per-block INT8 Q/K, keeps a block exact iff its score is at
+ * least mean + tau*std over the query block's row (the Sol rule), runs
+ * FlashAttention-style online softmax over the kept blocks only and adds one
+ * (1x64) or two (2x32) centroid terms for every skipped block
+ * ("Configure Sol Sparse Attention", How it works; The inputs that matter).
+ * A second entry point runs an explicit logical 128x128 block mask such as
+ * FlashVSR's LCSA streaming mask, with no centroids ("FlashVSR Sparge
+ * Attention", intro and How it works; "FlashVSR Kitchen Sparse Attention",
+ * intro).
+ *
+ * Conventions shared by every entry point
+ *  - Tensors are contiguous row-major: Q, O [B, H, Lq, d]; K, V [B, H, Lk, d].
+ *    bf16 buffers are passed as void pointers (raw IEEE bfloat16 bits).
+ *  - nQB = ceil(Lq/128) query blocks, nKB = ceil(Lk/64) key blocks,
+ *    nLK = ceil(Lk/128) logical key blocks of the mask entry.
+ *  - d is 64 or 128. n_prefix is a multiple of 128 (0 = no dense prefix).
+ *  - Device pointers only, 16-byte aligned; the caller owns every buffer,
+ *    including the workspace. The library never allocates, frees or
+ *    synchronises (bsva_check_status is the one call that synchronises).
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream) of the current device.
+ *  - Every call returns a status code. On a validation failure nothing is
+ *    launched and no output is touched; bsva_last_error() then holds a
+ *    message for the calling thread. There is no fallback path.
+ */
+#ifndef BSVA_H
+#define BSVA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BSVA_ABI_VERSION 1
+
+enum bsva_status {
+  BSVA_OK = 0,
+  BSVA_ERR_INVALID_ARG = 1,    /* null pointer, bad size, misalignment      */
+  BSVA_ERR_UNSUPPORTED = 2,    /* device is not sm_100, d not in {64, 128}  */
+  BSVA_ERR_WORKSPACE = 3,      /* workspace missing or too small            */
+  BSVA_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed      */
+  BSVA_ERR_DEVICE_TIMEOUT = 5  /* a bounded device-side wait gave up        */
+};
+
+typedef struct CUstream_st* bsva_stream_t;
+
+typedef struct bsva_shape {
+  int B, H;      /* batch, heads                                  */
+  int Lq, Lk;    /* query and key lengths (tokens)                */
+  int d;         /* head dim: 64 or 128                           */
+  int n_prefix;  /* leading tokens kept dense (multiple of 128)   */
+} bsva_shape;
+
+/* ABI version of the loaded library; loaders compare it with BSVA_ABI_VERSION
+ * ("FlashVSR Kitchen Sparse Attention", When it bites: ABI check on load). */
+int bsva_abi_version(void);
+
+/* Message for the last failed call on this thread ("" if none). The pointer
+ * stays valid until the next call on the same thread. */
+const char* bsva_last_error(void);
+
+/* Bytes of device workspace needed by sparse_attn_fwd (centroid_mode 1 or 2)
+ * or masked_block_attn_fwd (centroid_mode 0) for shape s; 0 on a bad shape.
+ * The first 256 bytes hold the device status word and must be zero before the
+ * first call (bsva_check_status clears them). */
+size_t bsva_workspace_bytes(bsva_shape s, int centroid_mode);
+
+/* Per-block symmetric INT8 quantisation and integer sum-pools, alone.
+ * ("Configure Sol Sparse Attention", How it works: the proxy and the exact
+ * path read the same prequantized INT8 Q/K.)
+ *   q, k      in : bf16 [B,H,Lq,d], [B,H,Lk,d]
+ *   q8, k8    out: int8, same shapes. Per block: s = fl32(amax/127),
+ *                  x8 = clamp(rint_half_even(fl32(x/s)), -127, 127); 0 if s = 0.
+ *   q_scale   out: fp32 [B,H,nQB]  (128-row Q blocks)
+ *   k_scale   out: fp32 [B,H,nKB]  (64-row K blocks)
+ *   q_pool    out: int32 [B,H,nQB,d]   column sums of each Q block's INT8 rows
+ *   k_pool    out: int32 [B,H,nKB,2,d] column sums of each 32-row half of
+ *                  each K block (a tail block's halves are rows [0,min(32,n))
+ *                  and [32,n); an empty half is 0).                          */
+int bsva_quantize_qk(bsva_shape s, const void* q, const void* k,
+                     int8_t* q8, float* q_scale, int8_t* k8, float* k_scale,
+                     int32_t* q_pool, int32_t* k_pool, bsva_stream_t stream);
+
+/* Quantise + proxy score + Sol routing ("Configure Sol Sparse Attention",
+ * How it works; The inputs that matter: routing_threshold, prefix_policy).
+ * Runs bsva_quantize_qk, then for every query-block row i:
+ *   s_ij = fl64(fl64(dot_ij * k_scale_j) / n_j),
+ *   dot_ij = sum_c q_pool_i[c] * (k_pool_j0[c] + k_pool_j1[c]) (exact int64),
+ *   mu, sigma = population mean and std of s_ij over the routed key blocks
+ *   (those starting at or after n_prefix), T = mu + tau*sigma, keep iff s >= T.
+ * Rows of query blocks starting before n_prefix, rows whose routed scores are
+ * all equal, and tau = -inf keep every block; key blocks before n_prefix are
+ * always kept.
+ *   tau        routing threshold (the pages' default is 1.0; -INFINITY = dense)
+ *   kept_mask  out: uint8 [B,H,nQB,nKB], 1 = exact
+ *   kept_idx   out: int32 [B,H,nQB,nKB], kept key-block indices ascending;
+ *                   entries at and after kept_cnt are unspecified
+ *   kept_cnt   out: int32 [B,H,nQB]
+ *   row_stats  out, nullable: fp64 [B,H,nQB,3] = (mu, sigma, T); T = -inf for
+ *                   rows that keep every block.                              */
+int sparse_attn_route(bsva_shape s, const void* q, const void* k, double tau,
+                      int8_t* q8, float* q_scale, int8_t* k8, float* k_scale,
+                      int32_t* q_pool, int32_t* k_pool,
+                      uint8_t* kept_mask, int32_t* kept_idx, int32_t* kept_cnt,
+                      double* row_stats, bsva_stream_t stream);
+
+/* Sparse attention over the routed blocks plus centroid terms
+ * ("Configure Sol Sparse Attention", How it works: skipped blocks are
+ * replaced by one 64-token centroid, or two 32-token centroids in 2x32 mode,
+ * inside the same online softmax).
+ *   Inputs are the outputs of sparse_attn_route (k_pool feeds the centroid
+ *   keys; v is bf16 [B,H,Lk,d]).
+ *   Exact term (row r, key t of kept block j): logit = sq_i*sk_j*scale*(q8_r . k8_t).
+ *   Centroid term (group g of skipped block j): kbar = sk_j*pool_g/|g|,
+ *     logit = sq_i*scale*(q8_r . kbar) + ln|g|, value = mean of V over g.
+ *   centroid_mode  1 = 1x64, 2 = 2x32
+ *   softmax_scale  <= 0 selects 1/sqrt(d)
+ *   out  out: bf16 [B,H,Lq,d]; lse out, nullable: fp32 [B,H,Lq] (natural log)
+ *   workspace      >= bsva_workspace_bytes(s, centroid_mode) bytes, 256-aligned */
+int sparse_attn_fwd(bsva_shape s, const int8_t* q8, const float* q_scale,
+                    const int8_t* k8, const float* k_scale,
+                    const int32_t* k_pool, const void* v,
+                    const uint8_t* kept_mask, const int32_t* kept_idx,
+                    const int32_t* kept_cnt, int centroid_mode,
+                    float softmax_scale, void* out, float* lse,
+                    void* workspace, size_t workspace_bytes,
+                    bsva_stream_t stream);
+
+/* Attention over an explicit logical block mask, exact terms only
+ * ("FlashVSR Sparge Attention", How it works: routing on logical
+ * 128-query x 128-key blocks, converted to the kernel's physical geometry
+ * after routing, one sparse call).
+ *   block_mask  uint8 [B, mask_heads, nQB, nLK]; mask_heads is 1 (shared by
+ *               all heads) or H. Physical 64-key block j of query block i runs
+ *               iff block_mask[b, h % mask_heads, i, j/2] != 0.
+ *   A query row with no allowed block gets out = 0 and lse = -inf.
+ *   workspace   >= bsva_workspace_bytes(s, 0) bytes, 256-aligned.
+ *   Other arguments as in sparse_attn_fwd.                                   */
+int masked_block_attn_fwd(bsva_shape s, const int8_t* q8, const float* q_scale,
+                          const int8_t* k8, const float* k_scale,
+                          const void* v, const uint8_t* block_mask,
+                          int mask_heads, float softmax_scale, void* out,
+                          float* lse, void* workspace, size_t workspace_bytes,
+                          bsva_stream_t stream);
+
+/* Synchronises `stream`, reads and clears the workspace's status word.
+ * Returns BSVA_OK, or BSVA_ERR_DEVICE_TIMEOUT if a kernel's bounded wait gave
+ * up since the last check (its outputs are then invalid). */
+int bsva_check_status(void* workspace, bsva_stream_t stream);
+
+/* Test hook for the failure path: launches one CTA that waits on a barrier
+ * nothing arrives at, with a wait bound of limit_ns nanoseconds
+ * (1e3 <= limit_ns <= 1e9). The wait runs out, the kernel records
+ * BSVA_ERR_DEVICE_TIMEOUT in the workspace status word and returns. */
+int bsva_selftest_timeout(void* workspace, size_t workspace_bytes,
+                          long long limit_ns, bsva_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSVA_H */

@@ -1,0 +1,161 @@
+"""Helpers for the GPU-vs-oracle parity tests (imported by tests only).
+
+The CUDA path and the oracle both start from the same seeded bf16 inputs
+(``workloads``); no value computed on the GPU is ever fed to the oracle.
+Bars (as the method is specified): INT8 tensors, scales, pools and the kept
+mask bit-exact, except routed blocks whose score lies within 1e-6*std of the
+threshold (counted); outputs within max-abs 1e-2 and relative L2 5e-3.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+import oracle
+import workloads
+
+ATOL = 1e-2
+REL_L2 = 5e-3
+LSE_ATOL = 1e-3
+
+
+@dataclass
+class Report:
+    band: int = 0                 # near-threshold routed blocks in the compared rows
+    band_mismatch: int = 0        # of which the GPU decided differently
+    rows_skipped: int = 0         # query blocks left out of the output check
+    max_abs: float = 0.0
+    rel_l2: float = 0.0
+    lse_max_abs: float = 0.0
+    notes: list = field(default_factory=list)
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().numpy()
+
+
+def inputs(w, device="cuda"):
+    Q, K, V = workloads.batch_qkv(w)
+    return Q.to(device), K.to(device), V.to(device)
+
+
+def head_np(w, b, h):
+    q, k, v = workloads.head_qkv(w, b, h)
+    return q.float().numpy(), k.float().numpy(), v.float().numpy()
+
+
+def check_quant(route, ref, b, h):
+    """INT8 tensors, scales and pools of one head, bit for bit."""
+    assert np.array_equal(to_np(route.q8[b, h]), ref["q8"]), "q8 differs"
+    assert np.array_equal(to_np(route.k8[b, h]), ref["k8"]), "k8 differs"
+    assert np.array_equal(to_np(route.q_scale[b, h]), ref["q_scale"]), "q_scale differs"
+    assert np.array_equal(to_np(route.k_scale[b, h]), ref["k_scale"]), "k_scale differs"
+    assert np.array_equal(to_np(route.q_pool[b, h]).astype(np.int64), ref["q_pool"]), "q_pool differs"
+    assert np.array_equal(to_np(route.k_pool[b, h]).astype(np.int64), ref["k_pool"]), "k_pool differs"
+
+
+def check_route(route, ref, b, h, rep: Report):
+    """Kept mask bit-exact outside the near-threshold band; lists consistent with the mask."""
+    gm = to_np(route.kept_mask[b, h]).astype(bool)
+    om = ref["keep"]
+    diff = gm != om
+    band = ref["band"]
+    rep.band += int(band.sum())
+    rep.band_mismatch += int((diff & band).sum())
+    bad = diff & ~band
+    assert not bad.any(), f"kept mask differs outside the band at {np.argwhere(bad)[:5].tolist()}"
+    cnt = to_np(route.kept_cnt[b, h])
+    idx = to_np(route.kept_idx[b, h])
+    assert np.array_equal(cnt, gm.sum(axis=1)), "kept_cnt != popcount(kept_mask)"
+    for i in range(gm.shape[0]):
+        assert np.array_equal(idx[i, :cnt[i]], np.nonzero(gm[i])[0]), f"kept_idx row {i}"
+    if route.row_stats is not None:
+        st = to_np(route.row_stats[b, h])
+        ref_st = ref["stats"]
+        fin = np.isfinite(ref_st[:, 2])
+        assert np.array_equal(np.isfinite(st[:, 2]), fin), "all-kept rows differ"
+        scale = np.abs(ref_st[:, 0]) + ref_st[:, 1] + 1e-300
+        assert (np.abs(st[:, 0] - ref_st[:, 0]) <= 1e-12 * scale).all(), "mu differs"
+        assert (np.abs(st[:, 1] - ref_st[:, 1]) <= 1e-12 * scale).all(), "sigma differs"
+    return diff
+
+
+def compare_rows(O_gpu, lse_gpu, O_ref, lse_ref, rows, rep: Report):
+    """Accumulate output error over the given row indices."""
+    if len(rows) == 0:
+        return
+    g = O_gpu[rows].astype(np.float64)
+    r = O_ref[rows]
+    err = np.abs(g - r)
+    rep.max_abs = max(rep.max_abs, float(err.max()))
+    num = float(np.sqrt((err ** 2).sum()))
+    den = float(np.sqrt((r ** 2).sum())) + 1e-300
+    rep.rel_l2 = max(rep.rel_l2, num / den)
+    if lse_gpu is not None:
+        lg, lr = lse_gpu[rows].astype(np.float64), lse_ref[rows]
+        both_inf = np.isneginf(lg) & np.isneginf(lr)
+        assert (np.isneginf(lg) == np.isneginf(lr)).all(), "empty-row lse differs"
+        if (~both_inf).any():
+            rep.lse_max_abs = max(rep.lse_max_abs, float(np.abs(lg[~both_inf] - lr[~both_inf]).max()))
+
+
+def assert_within(rep: Report, what: str):
+    assert rep.max_abs <= ATOL, f"{what}: max-abs {rep.max_abs:.3e} > {ATOL}"
+    assert rep.rel_l2 <= REL_L2, f"{what}: rel-L2 {rep.rel_l2:.3e} > {REL_L2}"
+    assert rep.lse_max_abs <= LSE_ATOL, f"{what}: lse max-abs {rep.lse_max_abs:.3e} > {LSE_ATOL}"
+
+
+def q_rows(Lq, blocks):
+    rows = []
+    for i in blocks:
+        rows.extend(range(128 * i, min(Lq, 128 * i + 128)))
+    return np.array(rows, dtype=np.int64)
+
+
+def sol_parity(bsva, w, tau, heads=None, q_blocks=None, centroid_mode=None):
+    """Route + fwd on the GPU over the whole workload; compare sampled heads/blocks with the oracle."""
+    mode = centroid_mode or w.centroid_mode
+    Q, K, V = inputs(w)
+    route = bsva.sparse_attn_route(Q, K, tau, n_prefix=w.n_prefix, row_stats=True)
+    out, lse = bsva.sparse_attn_fwd(route, V, mode, with_lse=True)
+    torch.cuda.synchronize()
+    heads = heads or [(b, h) for b in range(w.B) for h in range(w.H)]
+    rep = Report()
+    for b, h in heads:
+        q, k, v = head_np(w, b, h)
+        ref = oracle.route_head(q, k, tau, w.n_prefix)
+        check_quant(route, ref, b, h)
+        diff = check_route(route, ref, b, h, rep)
+        blocks = list(range(w.nQB)) if q_blocks is None else [i for i in q_blocks if i < w.nQB]
+        clean = [i for i in blocks if not diff[i].any()]
+        rep.rows_skipped += len(blocks) - len(clean)
+        O_ref, lse_ref = oracle.sol_attention_head(ref["q8"], ref["q_scale"], ref["k8"], ref["k_scale"], v,
+                                                   ref["keep"], mode, 0.0, q_blocks=clean)
+        compare_rows(to_np(out[b, h].float()), to_np(lse[b, h]), O_ref, lse_ref, q_rows(w.Lq, clean), rep)
+    return route, out, lse, rep
+
+
+def masked_parity(bsva, w, mask, heads=None, q_blocks=None, softmax_scale=0.0):
+    """Quantise on the GPU, run the mask entry, compare with the oracle's masked attention."""
+    Q, K, V = inputs(w)
+    qk = bsva.quantize_qk(Q, K)
+    m_dev = mask.to("cuda")
+    out, lse = bsva.masked_block_attn_fwd(qk["q8"], qk["q_scale"], qk["k8"], qk["k_scale"], V, m_dev,
+                                          softmax_scale=softmax_scale, with_lse=True)
+    torch.cuda.synchronize()
+    heads = heads or [(b, h) for b in range(w.B) for h in range(w.H)]
+    rep = Report()
+    Hm = mask.shape[1]
+    for b, h in heads:
+        q, k, v = head_np(w, b, h)
+        ref = oracle.route_head(q, k, -math.inf, 0)
+        assert np.array_equal(to_np(qk["q8"][b, h]), ref["q8"]) and np.array_equal(to_np(qk["k8"][b, h]), ref["k8"])
+        allowed = oracle.physical_allowed(mask[b, h % Hm].numpy(), w.nKB)
+        blocks = list(range(w.nQB)) if q_blocks is None else [i for i in q_blocks if i < w.nQB]
+        O_ref, lse_ref = oracle.masked_attention_head(ref["q8"], ref["q_scale"], ref["k8"], ref["k_scale"], v,
+                                                      allowed, softmax_scale, q_blocks=blocks)
+        compare_rows(to_np(out[b, h].float()), to_np(lse[b, h]), O_ref, lse_ref, q_rows(w.Lq, blocks), rep)
+    return out, lse, rep

@@ -1,0 +1,102 @@
+"""The C-ABI library loads, exports every symbol its header declares, and
+rejects bad arguments with status codes (CPU only: no kernel is launched)."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+import torch
+
+import block_sparse_video_int8_b200 as bsva
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "bsva.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(\w+)\s*\(", src, flags=re.M)))
+
+
+def test_library_builds_and_exports_every_declared_symbol():
+    from block_sparse_video_int8_b200 import build
+    build.build()
+    lib = ctypes.CDLL(bsva.lib_path())
+    names = _declared()
+    assert {"sparse_attn_route", "sparse_attn_fwd", "masked_block_attn_fwd", "bsva_quantize_qk",
+            "bsva_abi_version", "bsva_last_error", "bsva_workspace_bytes", "bsva_check_status",
+            "bsva_selftest_timeout"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_abi_version_matches_binding():
+    assert bsva.abi_version() == bsva.ABI_VERSION == 1
+
+
+def test_workspace_size_arithmetic():
+    s = bsva.Shape(1, 40, 32760, 32760, 128, 0)
+    nKB, nQB, BH = 512, 256, 40
+    n2 = bsva.workspace_bytes(s, 2)
+    nCT = math.ceil(nKB * 2 / 32)
+    assert n2 >= BH * nCT * 64 * 128 * 3 + BH * nCT * 32 * 8
+    n0 = bsva.workspace_bytes(s, 0)
+    assert n0 >= BH * nQB * nKB * 4
+    with pytest.raises(bsva.BsvaError):
+        bsva.workspace_bytes(bsva.Shape(1, 1, 100, 100, 96, 0), 1)   # d = 96
+    with pytest.raises(bsva.BsvaError):
+        bsva.workspace_bytes(s, 3)
+
+
+def _raw_route(shape, ptr=0):
+    lib = bsva.load()
+    P = ctypes.c_void_p(ptr) if ptr else None
+    return lib.sparse_attn_route(shape, P, P, ctypes.c_double(1.0), P, P, P, P, P, P, P, P, P, None,
+                                 None)
+
+
+def test_bad_arguments_return_codes_without_launching():
+    lib = bsva.load()
+    good = bsva.Shape(1, 2, 256, 256, 128, 0)
+    assert _raw_route(good) == 1                                   # NULL pointers
+    assert b"NULL" in lib.bsva_last_error()
+    assert _raw_route(bsva.Shape(1, 2, 256, 256, 80, 0), 0x1000) == 2   # d = 80 unsupported
+    assert _raw_route(bsva.Shape(1, 2, 256, 256, 128, 100), 0x1000) == 1  # prefix not /128
+    assert _raw_route(bsva.Shape(0, 2, 256, 256, 128, 0), 0x1000) == 1
+    assert _raw_route(good, 0x1001) == 1                           # misaligned
+    assert b"aligned" in lib.bsva_last_error()
+    # NaN / +inf tau are rejected before any device work
+    P = ctypes.c_void_p(0x1000)
+    rc = lib.sparse_attn_route(good, P, P, ctypes.c_double(float("nan")), P, P, P, P, P, P, P, P, P,
+                               None, None)
+    assert rc == 1
+
+
+def test_fwd_rejects_bad_mode_and_small_workspace():
+    lib = bsva.load()
+    s = bsva.Shape(1, 2, 256, 256, 128, 0)
+    P = ctypes.c_void_p(0x10000)
+    rc = lib.sparse_attn_fwd(s, P, P, P, P, P, P, P, P, P, 3, ctypes.c_float(0), P, None, P, 1 << 30, None)
+    assert rc == 1
+    rc = lib.sparse_attn_fwd(s, P, P, P, P, P, P, P, P, P, 1, ctypes.c_float(0), P, None, P, 16, None)
+    assert rc == 3
+    rc = lib.masked_block_attn_fwd(s, P, P, P, P, P, P, 3, ctypes.c_float(0), P, None, P, 1 << 30, None)
+    assert rc == 1                                                 # mask_heads not in {1, H}
+
+
+def test_no_device_is_an_error_not_a_fallback():
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    lib = bsva.load()
+    s = bsva.Shape(1, 2, 256, 256, 128, 0)
+    P = ctypes.c_void_p(0x10000)
+    rc = lib.bsva_quantize_qk(s, P, P, P, P, P, P, P, P, None)
+    assert rc in (2, 4)
+    assert lib.bsva_last_error()
+
+
+def test_binding_refuses_cpu_tensors():
+    q = torch.zeros((1, 1, 128, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        bsva.sparse_attn_route(q, q, 1.0)

@@ -1,0 +1,125 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Small workloads are compared in full (every head, every query block); the
+five method configurations run at full size in the launch configuration the
+bench times, and are compared on sampled heads (all rows of their routing,
+bit-exact) and sampled query blocks (attention outputs).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from parity import (Report, assert_within, compare_rows, head_np, inputs, masked_parity, q_rows,
+                    sol_parity, to_np)
+
+pytestmark = pytest.mark.gpu
+
+SMALL_SOL = [("ragged_pe", 0.5), ("ragged_pe", 1.0), ("ragged_pe_2x32", 1.0), ("ragged_d64", 0.5),
+             ("cross", 1.0), ("prefix_small", 1.0), ("tiny", 1.0)]
+
+
+@pytest.mark.parametrize("name,tau", SMALL_SOL)
+def test_sol_small_full_compare(gpu_lib, name, tau):
+    w = workloads.get(name)
+    _, _, _, rep = sol_parity(gpu_lib, w, tau)
+    assert_within(rep, f"{name} tau={tau}")
+    print(f"{name} tau={tau}: {rep}")
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_sol_dense_limit_tau_neginf(gpu_lib, mode):
+    w = workloads.get("ragged_pe")
+    route, out, lse, rep = sol_parity(gpu_lib, w, -math.inf, centroid_mode=mode)
+    assert bool((route.kept_mask == 1).all())
+    assert_within(rep, "tau=-inf")
+
+
+def test_sol_high_tau_centroid_heavy(gpu_lib):
+    w = workloads.get("ragged_pe_2x32")
+    route, out, lse, rep = sol_parity(gpu_lib, w, 2.5)
+    assert_within(rep, "tau=2.5")
+
+
+def test_masked_small_lcsa(gpu_lib):
+    w = workloads.get("lcsa_small")
+    _, _, rep = masked_parity(gpu_lib, w, workloads.block_mask(w))
+    assert_within(rep, "lcsa_small")
+
+
+def test_masked_per_head_random_mask_with_empty_rows(gpu_lib):
+    w = workloads.get("cross")
+    rng = np.random.default_rng(5)
+    m = (rng.random((w.B, w.H, w.nQB, w.nLK)) < 0.4).astype(np.uint8)
+    m[0, 1, 2, :] = 0                       # a query block with nothing allowed
+    m[1, 0, :, :] = 1                       # a head with everything allowed
+    out, lse, rep = masked_parity(gpu_lib, w, torch.from_numpy(m), softmax_scale=0.07)
+    assert_within(rep, "random per-head mask")
+    assert bool((out[0, 1, 256:384] == 0).all())
+    assert bool(torch.isneginf(lse[0, 1, 256:384]).all())
+
+
+def test_deterministic_repeat(gpu_lib):
+    w = workloads.get("ragged_pe_2x32")
+    Q, K, V = inputs(w)
+    r1 = gpu_lib.sparse_attn_route(Q, K, 1.0)
+    o1 = gpu_lib.sparse_attn_fwd(r1, V, 2).clone()
+    r2 = gpu_lib.sparse_attn_route(Q, K, 1.0)
+    o2 = gpu_lib.sparse_attn_fwd(r2, V, 2)
+    torch.cuda.synchronize()
+    assert torch.equal(r1.kept_mask, r2.kept_mask)
+    assert torch.equal(o1, o2)
+
+
+def test_device_timeout_is_reported_and_context_survives(gpu_lib):
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    gpu_lib.selftest_timeout(ws, 2_000_000)          # a 2 ms wait that nothing completes
+    with pytest.raises(gpu_lib.BsvaError) as e:
+        gpu_lib.check_status(ws)
+    assert e.value.code == 5
+    gpu_lib.check_status(ws)                         # cleared
+    w = workloads.get("ragged_d64")                  # the context still works
+    _, _, _, rep = sol_parity(gpu_lib, w, 0.5, heads=[(0, 0)])
+    assert_within(rep, "after timeout")
+
+
+def test_binding_rejects_bad_inputs(gpu_lib):
+    q = torch.zeros((1, 1, 256, 96), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(gpu_lib.BsvaError) as e:
+        gpu_lib.sparse_attn_route(q, q, 1.0)
+    assert e.value.code == 2
+    q = torch.zeros((1, 1, 256, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(gpu_lib.BsvaError):
+        gpu_lib.sparse_attn_route(q, q, 1.0, n_prefix=100)
+
+
+# ---------------------------------------------------------------- full size
+def _sample_blocks(nQB, n_extra=4, seed=0):
+    rng = np.random.default_rng(seed)
+    base = {0, 1, nQB // 2, nQB - 1}
+    base |= set(int(x) for x in rng.choice(nQB, size=n_extra, replace=False))
+    return sorted(base)
+
+
+@pytest.mark.slow
+def test_full_lcsa(gpu_lib):
+    w = workloads.get("lcsa")
+    heads = [(0, 0), (0, w.H - 1)]
+    _, _, rep = masked_parity(gpu_lib, w, workloads.block_mask(w), heads=heads,
+                              q_blocks=_sample_blocks(w.nQB))
+    assert_within(rep, "lcsa full")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,tau", [("wan13b", 1.0), ("wan14b", 0.5), ("wan14b", 1.0), ("wan14b", 1.5),
+                                      ("h3", 1.0)])
+def test_full_sol(gpu_lib, name, tau):
+    w = workloads.get(name)
+    heads = [(0, 0), (0, w.H - 1)]
+    _, _, _, rep = sol_parity(gpu_lib, w, tau, heads=heads, q_blocks=_sample_blocks(w.nQB))
+    print(f"{name} tau={tau}: {rep}")
+    assert_within(rep, f"{name} tau={tau}")
+    assert rep.band_mismatch <= max(2, rep.band)
