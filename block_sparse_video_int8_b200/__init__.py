@@ -24,11 +24,14 @@ __all__ = [
     "BsvaError", "load", "lib_path", "Route", "Shape", "abi_version",
     "workspace_bytes", "quantize_qk", "sparse_attn_route", "sparse_attn_fwd",
     "masked_block_attn_fwd", "check_status", "selftest_timeout", "new_workspace",
+    "build_centroids", "sparse_attn_core",
 ]
 
 ABI_VERSION = 1
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
+
+OUT_DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA",
           5: "DEVICE_TIMEOUT"}
@@ -58,9 +61,13 @@ _SIGS = {
     "sparse_attn_route": (ctypes.c_int, [Shape, _P, _P, ctypes.c_double, _P, _P, _P, _P, _P, _P,
                                          _P, _P, _P, _P, _P]),
     "sparse_attn_fwd": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int,
-                                       ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]),
+                                       ctypes.c_float, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
     "masked_block_attn_fwd": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, _P, ctypes.c_int,
-                                             ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]),
+                                             ctypes.c_float, ctypes.c_int, _P, _P, _P, ctypes.c_size_t,
+                                             _P]),
+    "bsva_build_centroids": (ctypes.c_int, [Shape, _P, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, _P]),
+    "bsva_sparse_attn_core": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int,
+                                             ctypes.c_float, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
     "bsva_check_status": (ctypes.c_int, [_P, _P]),
     "bsva_selftest_timeout": (ctypes.c_int, [_P, ctypes.c_size_t, ctypes.c_longlong, _P]),
 }
@@ -213,33 +220,71 @@ def sparse_attn_route(q: torch.Tensor, k: torch.Tensor, tau: float, n_prefix: in
     return out
 
 
+def _out(out, shape, out_dtype, device):
+    if out_dtype not in OUT_DTYPES:
+        raise TypeError(f"out_dtype must be torch.bfloat16 or torch.float32, got {out_dtype}")
+    if out is None:
+        return torch.empty(shape, dtype=out_dtype, device=device)
+    _need(out, out_dtype, shape, "out")
+    return out
+
+
 def sparse_attn_fwd(route: Route, v: torch.Tensor, centroid_mode: int, softmax_scale: float = 0.0,
                     with_lse: bool = False, workspace: torch.Tensor | None = None,
                     out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
-                    stream=None):
+                    out_dtype=torch.bfloat16, stream=None):
     """Sparse attention over the routed blocks plus centroids (C ABI ``sparse_attn_fwd``).
 
-    Returns ``out`` (bf16 [B, H, Lq, d]) or ``(out, lse)`` when ``with_lse``.
+    Returns ``out`` ([B, H, Lq, d], bf16 or fp32) or ``(out, lse)`` when ``with_lse``.
     """
     lib = load()
     s = route.shape
     _need(v, torch.bfloat16, (s.B, s.H, s.Lk, s.d), "v")
     if workspace is None:
         workspace = new_workspace(s, centroid_mode, v.device)
-    if out is None:
-        out = torch.empty((s.B, s.H, s.Lq, s.d), dtype=torch.bfloat16, device=v.device)
+    out = _out(out, (s.B, s.H, s.Lq, s.d), out_dtype, v.device)
     if with_lse and lse is None:
         lse = torch.empty((s.B, s.H, s.Lq), dtype=torch.float32, device=v.device)
     _check(lib.sparse_attn_fwd(s, _ptr(route.q8), _ptr(route.q_scale), _ptr(route.k8),
                                _ptr(route.k_scale), _ptr(route.k_pool), _ptr(v), _ptr(route.kept_mask),
                                _ptr(route.kept_idx), _ptr(route.kept_cnt), centroid_mode,
-                               ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace),
+                               ctypes.c_float(softmax_scale), OUT_DTYPES[out.dtype], _ptr(out), _ptr(lse),
+                               _ptr(workspace),
                                workspace.numel(), _stream(stream)))
     return (out, lse) if with_lse else out
 
 
+def build_centroids(route: Route, v: torch.Tensor, centroid_mode: int, workspace: torch.Tensor,
+                    stream=None):
+    """The centroid table of (k_pool, k_scale, v) into ``workspace`` (C ABI ``bsva_build_centroids``)."""
+    lib = load()
+    s = route.shape
+    _need(v, torch.bfloat16, (s.B, s.H, s.Lk, s.d), "v")
+    _check(lib.bsva_build_centroids(s, _ptr(route.k_pool), _ptr(route.k_scale), _ptr(v), centroid_mode,
+                                    _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def sparse_attn_core(route: Route, v: torch.Tensor, centroid_mode: int, workspace: torch.Tensor,
+                     out: torch.Tensor, softmax_scale: float = 0.0, lse: torch.Tensor | None = None,
+                     stream=None):
+    """The attention kernel alone, on a workspace that holds the centroid table
+    (C ABI ``bsva_sparse_attn_core``)."""
+    lib = load()
+    s = route.shape
+    _need(v, torch.bfloat16, (s.B, s.H, s.Lk, s.d), "v")
+    if out.dtype not in OUT_DTYPES:
+        raise TypeError("out must be bf16 or fp32")
+    _need(out, out.dtype, (s.B, s.H, s.Lq, s.d), "out")
+    _check(lib.bsva_sparse_attn_core(s, _ptr(route.q8), _ptr(route.q_scale), _ptr(route.k8), _ptr(route.k_scale),
+                                     _ptr(v), _ptr(route.kept_mask), _ptr(route.kept_idx), _ptr(route.kept_cnt),
+                                     centroid_mode, ctypes.c_float(softmax_scale), OUT_DTYPES[out.dtype],
+                                     _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
 def masked_block_attn_fwd(q8, q_scale, k8, k_scale, v, block_mask, softmax_scale: float = 0.0,
-                          with_lse: bool = False, workspace=None, out=None, lse=None, stream=None):
+                          with_lse: bool = False, workspace=None, out=None, lse=None,
+                          out_dtype=torch.bfloat16, stream=None):
     """Attention over an explicit logical 128x128 block mask (C ABI ``masked_block_attn_fwd``)."""
     lib = load()
     B, H, Lq, d = q8.shape
@@ -254,13 +299,13 @@ def masked_block_attn_fwd(q8, q_scale, k8, k_scale, v, block_mask, softmax_scale
     mask_heads = block_mask.shape[1]
     if workspace is None:
         workspace = new_workspace(s, 0, v.device)
-    if out is None:
-        out = torch.empty((B, H, Lq, d), dtype=torch.bfloat16, device=v.device)
+    out = _out(out, (B, H, Lq, d), out_dtype, v.device)
     if with_lse and lse is None:
         lse = torch.empty((B, H, Lq), dtype=torch.float32, device=v.device)
     _check(lib.masked_block_attn_fwd(s, _ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(k_scale), _ptr(v),
                                      _ptr(block_mask), mask_heads, ctypes.c_float(softmax_scale),
-                                     _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+                                     OUT_DTYPES[out.dtype], _ptr(out), _ptr(lse), _ptr(workspace),
+                                     workspace.numel(),
                                      _stream(stream)))
     return (out, lse) if with_lse else out
 

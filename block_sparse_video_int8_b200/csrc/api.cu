@@ -122,8 +122,8 @@ int check_workspace(void* ws, size_t bytes, size_t need) {
 // Shared tail of both attention entry points.
 int run_attention(const bsva_shape& s, const int8_t* q8, const float* q_scale, const int8_t* k8,
                   const float* k_scale, const void* v, const uint8_t* kept_mask, const int32_t* kept_idx,
-                  const int32_t* kept_cnt, int centroid_mode, float softmax_scale, void* out, float* lse,
-                  unsigned char* ws, const WsLayout& L, cudaStream_t st) {
+                  const int32_t* kept_cnt, int centroid_mode, float softmax_scale, int out_dtype, void* out,
+                  float* lse, unsigned char* ws, const WsLayout& L, cudaStream_t st) {
   int rc = get_encoder();
   if (rc) return rc;
   const uint64_t BH = uint64_t(s.B) * s.H;
@@ -161,7 +161,8 @@ int run_attention(const bsva_shape& s, const int8_t* q8, const float* q_scale, c
   a.cfac = centroid_mode > 0 ? reinterpret_cast<const float*>(ws + L.cfac) : nullptr;
   a.cbias = centroid_mode > 0 ? reinterpret_cast<const float*>(ws + L.cbias) : nullptr;
   a.order = nullptr;
-  a.out = reinterpret_cast<__nv_bfloat16*>(out);
+  a.out = out_dtype == BSVA_OUT_BF16 ? reinterpret_cast<__nv_bfloat16*>(out) : nullptr;
+  a.out_f32 = out_dtype == BSVA_OUT_F32 ? reinterpret_cast<float*>(out) : nullptr;
   a.lse = lse;
   a.status = reinterpret_cast<uint32_t*>(ws + L.status);
   a.wait_limit_ns = kWaitLimitNs;
@@ -222,43 +223,112 @@ int sparse_attn_route(bsva_shape s, const void* q, const void* k, double tau, in
   return ok();
 }
 
-int sparse_attn_fwd(bsva_shape s, const int8_t* q8, const float* q_scale, const int8_t* k8, const float* k_scale,
-                    const int32_t* k_pool, const void* v, const uint8_t* kept_mask, const int32_t* kept_idx,
-                    const int32_t* kept_cnt, int centroid_mode, float softmax_scale, void* out, float* lse,
-                    void* workspace, size_t workspace_bytes, bsva_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+int check_fwd_args(const bsva_shape& s, const int8_t* q8, const float* q_scale, const int8_t* k8,
+                   const float* k_scale, const void* v, const uint8_t* kept_mask, const int32_t* kept_idx,
+                   const int32_t* kept_cnt, int centroid_mode, float softmax_scale, int out_dtype, void* out,
+                   float* lse) {
   int rc;
   if ((rc = check_shape(s))) return rc;
   if (centroid_mode != 1 && centroid_mode != 2)
     return fail(BSVA_ERR_INVALID_ARG, "centroid_mode = %d; use 1 (1x64) or 2 (2x32)", centroid_mode);
   if (std::isnan(softmax_scale) || std::isinf(softmax_scale))
     return fail(BSVA_ERR_INVALID_ARG, "softmax_scale must be finite");
+  if (out_dtype != BSVA_OUT_BF16 && out_dtype != BSVA_OUT_F32)
+    return fail(BSVA_ERR_INVALID_ARG, "out_dtype = %d; use BSVA_OUT_BF16 (0) or BSVA_OUT_F32 (1)", out_dtype);
   REQUIRE_PTR(q8, 16); REQUIRE_PTR(q_scale, 4); REQUIRE_PTR(k8, 16); REQUIRE_PTR(k_scale, 4);
-  REQUIRE_PTR(k_pool, 16); REQUIRE_PTR(v, 16); REQUIRE_PTR(kept_mask, 1); REQUIRE_PTR(kept_idx, 4);
+  REQUIRE_PTR(v, 16); REQUIRE_PTR(kept_mask, 1); REQUIRE_PTR(kept_idx, 4);
   REQUIRE_PTR(kept_cnt, 4); REQUIRE_PTR(out, 16);
   if (lse && !aligned(lse, 4)) return fail(BSVA_ERR_INVALID_ARG, "lse is not 4-byte aligned");
+  return BSVA_OK;
+}
+
+int check_centroid_args(const bsva_shape& s, const int32_t* k_pool, const float* k_scale, const void* v,
+                        int centroid_mode) {
+  int rc;
+  if ((rc = check_shape(s))) return rc;
+  if (centroid_mode != 1 && centroid_mode != 2)
+    return fail(BSVA_ERR_INVALID_ARG, "centroid_mode = %d; use 1 (1x64) or 2 (2x32)", centroid_mode);
+  REQUIRE_PTR(k_pool, 16); REQUIRE_PTR(k_scale, 4); REQUIRE_PTR(v, 16);
+  return BSVA_OK;
+}
+
+int build_centroids(const bsva_shape& s, const int32_t* k_pool, const float* k_scale, const void* v,
+                    int centroid_mode, unsigned char* ws, const WsLayout& L, cudaStream_t st) {
+  cudaError_t e = launch_centroids(s, centroid_mode, L.nCT, k_pool, k_scale, reinterpret_cast<const __nv_bfloat16*>(v),
+                                   reinterpret_cast<int8_t*>(ws + L.ck8), reinterpret_cast<__nv_bfloat16*>(ws + L.cv),
+                                   reinterpret_cast<float*>(ws + L.cfac), reinterpret_cast<float*>(ws + L.cbias), st);
+  if (e != cudaSuccess) return cuda_fail(e, "centroid launch");
+  return BSVA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int bsva_build_centroids(bsva_shape s, const int32_t* k_pool, const float* k_scale, const void* v,
+                         int centroid_mode, void* workspace, size_t workspace_bytes, bsva_stream_t stream) {
+  int rc;
+  if ((rc = check_centroid_args(s, k_pool, k_scale, v, centroid_mode))) return rc;
+  const WsLayout L = ws_layout(s, centroid_mode);
+  if ((rc = check_workspace(workspace, workspace_bytes, L.total))) return rc;
+  if ((rc = check_device())) return rc;
+  if ((rc = build_centroids(s, k_pool, k_scale, v, centroid_mode, static_cast<unsigned char*>(workspace), L,
+                            reinterpret_cast<cudaStream_t>(stream))))
+    return rc;
+  return ok();
+}
+
+int bsva_sparse_attn_core(bsva_shape s, const int8_t* q8, const float* q_scale, const int8_t* k8,
+                          const float* k_scale, const void* v, const uint8_t* kept_mask, const int32_t* kept_idx,
+                          const int32_t* kept_cnt, int centroid_mode, float softmax_scale, int out_dtype, void* out,
+                          float* lse, void* workspace, size_t workspace_bytes, bsva_stream_t stream) {
+  int rc;
+  if ((rc = check_fwd_args(s, q8, q_scale, k8, k_scale, v, kept_mask, kept_idx, kept_cnt, centroid_mode,
+                           softmax_scale, out_dtype, out, lse)))
+    return rc;
+  const WsLayout L = ws_layout(s, centroid_mode);
+  if ((rc = check_workspace(workspace, workspace_bytes, L.total))) return rc;
+  if ((rc = check_device())) return rc;
+  return run_attention(s, q8, q_scale, k8, k_scale, v, kept_mask, kept_idx, kept_cnt, centroid_mode, softmax_scale,
+                       out_dtype, out, lse, static_cast<unsigned char*>(workspace), L,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+int sparse_attn_fwd(bsva_shape s, const int8_t* q8, const float* q_scale, const int8_t* k8, const float* k_scale,
+                    const int32_t* k_pool, const void* v, const uint8_t* kept_mask, const int32_t* kept_idx,
+                    const int32_t* kept_cnt, int centroid_mode, float softmax_scale, int out_dtype, void* out,
+                    float* lse, void* workspace, size_t workspace_bytes, bsva_stream_t stream) {
+  int rc;
+  if ((rc = check_fwd_args(s, q8, q_scale, k8, k_scale, v, kept_mask, kept_idx, kept_cnt, centroid_mode,
+                           softmax_scale, out_dtype, out, lse)))
+    return rc;
+  REQUIRE_PTR(k_pool, 16);
   const WsLayout L = ws_layout(s, centroid_mode);
   if ((rc = check_workspace(workspace, workspace_bytes, L.total))) return rc;
   if ((rc = check_device())) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
-  cudaError_t e = launch_centroids(s, centroid_mode, L.nCT, k_pool, k_scale, reinterpret_cast<const __nv_bfloat16*>(v),
-                                   reinterpret_cast<int8_t*>(ws + L.ck8), reinterpret_cast<__nv_bfloat16*>(ws + L.cv),
-                                   reinterpret_cast<float*>(ws + L.cfac), reinterpret_cast<float*>(ws + L.cbias), st);
-  if (e != cudaSuccess) return cuda_fail(e, "centroid launch");
+  if ((rc = build_centroids(s, k_pool, k_scale, v, centroid_mode, ws, L, st))) return rc;
   return run_attention(s, q8, q_scale, k8, k_scale, v, kept_mask, kept_idx, kept_cnt, centroid_mode, softmax_scale,
-                       out, lse, ws, L, st);
+                       out_dtype, out, lse, ws, L, st);
 }
 
 int masked_block_attn_fwd(bsva_shape s, const int8_t* q8, const float* q_scale, const int8_t* k8,
                           const float* k_scale, const void* v, const uint8_t* block_mask, int mask_heads,
-                          float softmax_scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
-                          bsva_stream_t stream) {
+                          float softmax_scale, int out_dtype, void* out, float* lse, void* workspace,
+                          size_t workspace_bytes, bsva_stream_t stream) {
   int rc;
   if ((rc = check_shape(s))) return rc;
   if (mask_heads != 1 && mask_heads != s.H)
     return fail(BSVA_ERR_INVALID_ARG, "mask_heads = %d must be 1 or H = %d", mask_heads, s.H);
   if (std::isnan(softmax_scale) || std::isinf(softmax_scale))
     return fail(BSVA_ERR_INVALID_ARG, "softmax_scale must be finite");
+  if (out_dtype != BSVA_OUT_BF16 && out_dtype != BSVA_OUT_F32)
+    return fail(BSVA_ERR_INVALID_ARG, "out_dtype = %d; use BSVA_OUT_BF16 (0) or BSVA_OUT_F32 (1)", out_dtype);
   REQUIRE_PTR(q8, 16); REQUIRE_PTR(q_scale, 4); REQUIRE_PTR(k8, 16); REQUIRE_PTR(k_scale, 4);
   REQUIRE_PTR(v, 16); REQUIRE_PTR(block_mask, 1); REQUIRE_PTR(out, 16);
   if (lse && !aligned(lse, 4)) return fail(BSVA_ERR_INVALID_ARG, "lse is not 4-byte aligned");
@@ -271,7 +341,8 @@ int masked_block_attn_fwd(bsva_shape s, const int8_t* q8, const float* q_scale, 
   int32_t* kcnt = reinterpret_cast<int32_t*>(ws + L.kcnt);
   cudaError_t e = launch_mask_expand(s, block_mask, mask_heads, kidx, kcnt, st);
   if (e != cudaSuccess) return cuda_fail(e, "mask expansion launch");
-  return run_attention(s, q8, q_scale, k8, k_scale, v, nullptr, kidx, kcnt, 0, softmax_scale, out, lse, ws, L, st);
+  return run_attention(s, q8, q_scale, k8, k_scale, v, nullptr, kidx, kcnt, 0, softmax_scale, out_dtype, out, lse,
+                       ws, L, st);
 }
 
 int bsva_check_status(void* workspace, bsva_stream_t stream) {

@@ -78,8 +78,10 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (N == 0) {   // nothing to attend: o = 0, lse = -inf
     if (tid < QB && q0 + tid < a.Lq) {
-      uint4* o = reinterpret_cast<uint4*>(a.out + (size_t(bh) * a.Lq + q0 + tid) * D);
-      for (int c = 0; c < D / 8; ++c) o[c] = make_uint4(0, 0, 0, 0);
+      const size_t orow = (size_t(bh) * a.Lq + q0 + tid) * D;
+      uint4* o = a.out_f32 ? reinterpret_cast<uint4*>(a.out_f32 + orow) : reinterpret_cast<uint4*>(a.out + orow);
+      const int n16 = a.out_f32 ? D / 4 : D / 8;
+      for (int c = 0; c < n16; ++c) o[c] = make_uint4(0, 0, 0, 0);
       if (a.lse) a.lse[size_t(bh) * a.Lq + q0 + tid] = -INFINITY;
     }
     return;
@@ -288,19 +290,21 @@ __global__ void __launch_bounds__(kThreads, 2)
 
       uint32_t pk[32];
       float lsum = 0.f;
+      // The row sum adds the bf16-rounded weights that the PV product uses, so
+      // numerator and denominator see the same probabilities.
       if (exact) {
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const float p0 = ex2(x[2 * c] - m_use), p1 = ex2(x[2 * c + 1] - m_use);
-          lsum += p0 + p1;
           pk[c] = pack_bf16x2(p0, p1);
+          lsum += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xFFFF0000u);
         }
       } else {
 #pragma unroll
         for (int g = 0; g < 32; ++g) {
           const float p = ex2(x[g] - m_use);
-          lsum += p;
           pk[g] = pack_bf16x2(p, p);
+          lsum += __uint_as_float(pk[g] << 16);
         }
       }
       l += lsum;
@@ -315,21 +319,29 @@ __global__ void __launch_bounds__(kThreads, 2)
       tc_fence_after();
       const int qr = q0 + r;
       const float inv_l = l > 0.f ? 1.0f / l : 0.f;
-      __nv_bfloat16* orow = a.out + (size_t(bh) * a.Lq + qr) * D;
+      const size_t orow = (size_t(bh) * a.Lq + qr) * D;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t o[32];
         tmem_ld32(tmem + lane_base + O_COL + c0, o);
         tmem_wait_ld();
         if (qr < a.Lq) {
-          uint4 w[4];
-          uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+          if (a.out_f32) {
+            float4* dst = reinterpret_cast<float4*>(a.out_f32 + orow + c0);
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
-            wp[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+            for (int c = 0; c < 8; ++c)
+              dst[c] = make_float4(__uint_as_float(o[4 * c]) * inv_l, __uint_as_float(o[4 * c + 1]) * inv_l,
+                                   __uint_as_float(o[4 * c + 2]) * inv_l, __uint_as_float(o[4 * c + 3]) * inv_l);
+          } else {
+            uint4 w[4];
+            uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) dst[c] = w[c];
+            for (int c = 0; c < 16; ++c)
+              wp[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
+            uint4* dst = reinterpret_cast<uint4*>(a.out + orow + c0);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) dst[c] = w[c];
+          }
         }
       }
       if (a.lse && qr < a.Lq)

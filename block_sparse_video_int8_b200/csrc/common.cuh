@@ -274,7 +274,8 @@ struct AttnArgs {
   const float* cfac;        // [BH, nCT*32]
   const float* cbias;       // [BH, nCT*32]
   const int32_t* order;     // [BH*nQB] work order
-  __nv_bfloat16* out;       // [BH, Lq, d]
+  __nv_bfloat16* out;       // [BH, Lq, d] bf16 output, or
+  float* out_f32;           // [BH, Lq, d] fp32 output (exactly one is non-null)
   float* lse;               // [BH, Lq] nullable
   uint32_t* status;
   uint64_t wait_limit_ns;

@@ -48,6 +48,12 @@ enum bsva_status {
   BSVA_ERR_DEVICE_TIMEOUT = 5  /* a bounded device-side wait gave up        */
 };
 
+/* Element type of the attention output `out`. */
+enum bsva_out_dtype {
+  BSVA_OUT_BF16 = 0,   /* bf16 [B,H,Lq,d]                                   */
+  BSVA_OUT_F32 = 1     /* fp32 [B,H,Lq,d]; bf16 output equals its rounding  */
+};
+
 typedef struct CUstream_st* bsva_stream_t;
 
 typedef struct bsva_shape {
@@ -121,16 +127,39 @@ int sparse_attn_route(bsva_shape s, const void* q, const void* k, double tau,
  *     logit = sq_i*scale*(q8_r . kbar) + ln|g|, value = mean of V over g.
  *   centroid_mode  1 = 1x64, 2 = 2x32
  *   softmax_scale  <= 0 selects 1/sqrt(d)
- *   out  out: bf16 [B,H,Lq,d]; lse out, nullable: fp32 [B,H,Lq] (natural log)
+ *   out_dtype      BSVA_OUT_BF16 or BSVA_OUT_F32 (element type of out)
+ *   out  out: [B,H,Lq,d]; lse out, nullable: fp32 [B,H,Lq] (natural log)
  *   workspace      >= bsva_workspace_bytes(s, centroid_mode) bytes, 256-aligned */
 int sparse_attn_fwd(bsva_shape s, const int8_t* q8, const float* q_scale,
                     const int8_t* k8, const float* k_scale,
                     const int32_t* k_pool, const void* v,
                     const uint8_t* kept_mask, const int32_t* kept_idx,
                     const int32_t* kept_cnt, int centroid_mode,
-                    float softmax_scale, void* out, float* lse,
+                    float softmax_scale, int out_dtype, void* out, float* lse,
                     void* workspace, size_t workspace_bytes,
                     bsva_stream_t stream);
+
+/* The two halves of sparse_attn_fwd, for callers that reuse one K/V (and so
+ * one centroid table) across several query batches, or that time the phases:
+ * sparse_attn_fwd(...) launches exactly bsva_build_centroids(...) followed by
+ * bsva_sparse_attn_core(...).
+ * bsva_build_centroids writes the centroid table of (k_pool, k_scale, v) into
+ * the workspace: per group, the INT8 key rows (hi, lo) with pool = 128*hi + lo,
+ * the value rows (bf16(vbar), bf16(vbar - bf16(vbar))), sk_j/|g| and log2|g|.
+ * bsva_sparse_attn_core runs the attention kernel and reads that table; its
+ * arguments mean what they mean for sparse_attn_fwd.                        */
+int bsva_build_centroids(bsva_shape s, const int32_t* k_pool,
+                         const float* k_scale, const void* v, int centroid_mode,
+                         void* workspace, size_t workspace_bytes,
+                         bsva_stream_t stream);
+
+int bsva_sparse_attn_core(bsva_shape s, const int8_t* q8, const float* q_scale,
+                          const int8_t* k8, const float* k_scale, const void* v,
+                          const uint8_t* kept_mask, const int32_t* kept_idx,
+                          const int32_t* kept_cnt, int centroid_mode,
+                          float softmax_scale, int out_dtype, void* out,
+                          float* lse, void* workspace, size_t workspace_bytes,
+                          bsva_stream_t stream);
 
 /* Attention over an explicit logical block mask, exact terms only
  * ("FlashVSR Sparge Attention", How it works: routing on logical
@@ -145,8 +174,9 @@ int sparse_attn_fwd(bsva_shape s, const int8_t* q8, const float* q_scale,
 int masked_block_attn_fwd(bsva_shape s, const int8_t* q8, const float* q_scale,
                           const int8_t* k8, const float* k_scale,
                           const void* v, const uint8_t* block_mask,
-                          int mask_heads, float softmax_scale, void* out,
-                          float* lse, void* workspace, size_t workspace_bytes,
+                          int mask_heads, float softmax_scale, int out_dtype,
+                          void* out, float* lse, void* workspace,
+                          size_t workspace_bytes,
                           bsva_stream_t stream);
 
 /* Synchronises `stream`, reads and clears the workspace's status word.

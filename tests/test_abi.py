@@ -77,11 +77,13 @@ def test_fwd_rejects_bad_mode_and_small_workspace():
     lib = bsva.load()
     s = bsva.Shape(1, 2, 256, 256, 128, 0)
     P = ctypes.c_void_p(0x10000)
-    rc = lib.sparse_attn_fwd(s, P, P, P, P, P, P, P, P, P, 3, ctypes.c_float(0), P, None, P, 1 << 30, None)
+    rc = lib.sparse_attn_fwd(s, P, P, P, P, P, P, P, P, P, 3, ctypes.c_float(0), 0, P, None, P, 1 << 30, None)
     assert rc == 1
-    rc = lib.sparse_attn_fwd(s, P, P, P, P, P, P, P, P, P, 1, ctypes.c_float(0), P, None, P, 16, None)
+    rc = lib.sparse_attn_fwd(s, P, P, P, P, P, P, P, P, P, 1, ctypes.c_float(0), 0, P, None, P, 16, None)
     assert rc == 3
-    rc = lib.masked_block_attn_fwd(s, P, P, P, P, P, P, 3, ctypes.c_float(0), P, None, P, 1 << 30, None)
+    rc = lib.sparse_attn_fwd(s, P, P, P, P, P, P, P, P, P, 1, ctypes.c_float(0), 7, P, None, P, 1 << 30, None)
+    assert rc == 1                                                 # unknown out_dtype
+    rc = lib.masked_block_attn_fwd(s, P, P, P, P, P, P, 3, ctypes.c_float(0), 0, P, None, P, 1 << 30, None)
     assert rc == 1                                                 # mask_heads not in {1, H}
 
 

@@ -59,6 +59,7 @@ def test_masked_per_head_random_mask_with_empty_rows(gpu_lib):
     out, lse, rep = masked_parity(gpu_lib, w, torch.from_numpy(m), softmax_scale=0.07)
     assert_within(rep, "random per-head mask")
     assert bool((out[0, 1, 256:384] == 0).all())
+    assert bool((out[0, 1, :256] != 0).any())
     assert bool(torch.isneginf(lse[0, 1, 256:384]).all())
 
 
