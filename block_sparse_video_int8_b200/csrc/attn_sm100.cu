@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint8_t* kmask = a.kept_mask ? a.kept_mask + row_item * a.nKB : nullptr;
     const float* cfac = a.cfac + size_t(bh) * a.nCT * 32;
     const float* cbias = a.cbias + size_t(bh) * a.nCT * 32;
-    float m_ref = -INFINITY, l = 0.f;
+    float m_ref = -INFINITY, l = 0.f, le = 0.f;
     bool alive = true;
 
     for (int n = 0; n < N; ++n) {
@@ -284,20 +284,24 @@ __global__ void __launch_bounds__(kThreads, 2)
           tmem_wait_st();
         }
         l *= alpha;
+        le *= alpha;
         m_ref = m_new;
       }
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
 
       uint32_t pk[32];
       float lsum = 0.f;
-      // The row sum adds the bf16-rounded weights that the PV product uses, so
-      // numerator and denominator see the same probabilities.
+      // Two row sums: lb adds the bf16-rounded weights that the PV product uses
+      // (numerator and denominator then see the same probabilities), le adds
+      // the unrounded weights for the log-sum-exp.
+      float esum = 0.f;
       if (exact) {
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const float p0 = ex2(x[2 * c] - m_use), p1 = ex2(x[2 * c + 1] - m_use);
           pk[c] = pack_bf16x2(p0, p1);
           lsum += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xFFFF0000u);
+          esum += p0 + p1;
         }
       } else {
 #pragma unroll
@@ -305,9 +309,11 @@ __global__ void __launch_bounds__(kThreads, 2)
           const float p = ex2(x[g] - m_use);
           pk[g] = pack_bf16x2(p, p);
           lsum += __uint_as_float(pk[g] << 16);
+          esum += p;
         }
       }
       l += lsum;
+      le += esum;
       tmem_st32(tmem + lane_base + sc, pk);
       tmem_wait_st();
       tc_fence_before();
@@ -345,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
       if (a.lse && qr < a.Lq)
-        a.lse[size_t(bh) * a.Lq + qr] = l > 0.f ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+        a.lse[size_t(bh) * a.Lq + qr] = le > 0.f ? (m_ref + __log2f(le)) * 0.69314718055994531f : -INFINITY;
     }
   }
 
