@@ -68,6 +68,8 @@ _SIGS = {
     "bsva_build_centroids": (ctypes.c_int, [Shape, _P, _P, _P, ctypes.c_int, _P, ctypes.c_size_t, _P]),
     "bsva_sparse_attn_core": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int,
                                              ctypes.c_float, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
+    "masked_block_attn_fwd_noalloc": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, _P, ctypes.c_int,
+                                                     ctypes.c_float, ctypes.c_int, _P, _P, _P]),
     "bsva_check_status": (ctypes.c_int, [_P, _P]),
     "bsva_selftest_timeout": (ctypes.c_int, [_P, ctypes.c_size_t, ctypes.c_longlong, _P]),
 }

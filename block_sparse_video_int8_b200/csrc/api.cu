@@ -376,3 +376,84 @@ int bsva_selftest_timeout(void* workspace, size_t workspace_bytes, long long lim
 }
 
 }  // extern "C"
+
+// --------------------------------------------------- no-allocation variant --
+// masked_block_attn_fwd for callers that cannot allocate device memory: the
+// kept-block lists live in a scratch array compiled into this library instead
+// of a caller workspace. Layout of the array: [0, 256) status word,
+// [256, 256 + 4*kNoAllocMaxRows) kept counts, then the kept lists.
+namespace {
+
+constexpr size_t kNoAllocMaxRows = size_t(1) << 16;       // B*H*nQB
+constexpr size_t kNoAllocMaxEntries = size_t(1) << 21;    // B*H*nQB*nKB
+constexpr size_t kNoAllocCntOff = 256;
+constexpr size_t kNoAllocIdxOff = kNoAllocCntOff + 4 * kNoAllocMaxRows;
+constexpr size_t kNoAllocBytes = kNoAllocIdxOff + 4 * kNoAllocMaxEntries;   // 8,651,008 bytes
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once
+// per device (host code cannot use the array's name as a device address).
+int noalloc_scratch(unsigned char** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(BSVA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = static_cast<unsigned char*>(g_noalloc_ptr[dev]);
+  return BSVA_OK;
+}
+
+}  // namespace
+
+extern "C" int masked_block_attn_fwd_noalloc(bsva_shape s, const int8_t* q8, const float* q_scale, const int8_t* k8,
+                                             const float* k_scale, const void* v, const uint8_t* block_mask,
+                                             int mask_heads, float softmax_scale, int out_dtype, void* out,
+                                             float* lse, bsva_stream_t stream) {
+  int rc;
+  if ((rc = check_shape(s))) return rc;
+  if (mask_heads != 1 && mask_heads != s.H)
+    return fail(BSVA_ERR_INVALID_ARG, "mask_heads = %d must be 1 or H = %d", mask_heads, s.H);
+  if (std::isnan(softmax_scale) || std::isinf(softmax_scale))
+    return fail(BSVA_ERR_INVALID_ARG, "softmax_scale must be finite");
+  if (out_dtype != BSVA_OUT_BF16 && out_dtype != BSVA_OUT_F32)
+    return fail(BSVA_ERR_INVALID_ARG, "out_dtype = %d; use BSVA_OUT_BF16 (0) or BSVA_OUT_F32 (1)", out_dtype);
+  REQUIRE_PTR(q8, 16); REQUIRE_PTR(q_scale, 4); REQUIRE_PTR(k8, 16); REQUIRE_PTR(k_scale, 4);
+  REQUIRE_PTR(v, 16); REQUIRE_PTR(block_mask, 1); REQUIRE_PTR(out, 16);
+  if (lse && !aligned(lse, 4)) return fail(BSVA_ERR_INVALID_ARG, "lse is not 4-byte aligned");
+  const size_t nQB = (size_t(s.Lq) + QB - 1) / QB, nKB = (size_t(s.Lk) + KB - 1) / KB;
+  const size_t rows = size_t(s.B) * s.H * nQB;
+  if (rows > kNoAllocMaxRows || rows * nKB > kNoAllocMaxEntries)
+    return fail(BSVA_ERR_WORKSPACE,
+                "shape needs %zu kept-list rows and %zu entries; the built-in scratch holds at most %zu rows and "
+                "%zu entries (use masked_block_attn_fwd with a caller workspace)",
+                rows, rows * nKB, kNoAllocMaxRows, kNoAllocMaxEntries);
+  if ((rc = check_device())) return rc;
+  unsigned char* ws = nullptr;
+  if ((rc = noalloc_scratch(&ws))) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // the status word must start at zero; the lists are fully rewritten below
+  cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the scratch status word");
+  WsLayout L;
+  L.status = 0;
+  L.kcnt = kNoAllocCntOff;
+  L.kidx = kNoAllocIdxOff;
+  L.total = kNoAllocBytes;
+  int32_t* kidx = reinterpret_cast<int32_t*>(ws + L.kidx);
+  int32_t* kcnt = reinterpret_cast<int32_t*>(ws + L.kcnt);
+  e = launch_mask_expand(s, block_mask, mask_heads, kidx, kcnt, st);
+  if (e != cudaSuccess) return cuda_fail(e, "mask expansion launch");
+  return run_attention(s, q8, q_scale, k8, k_scale, v, nullptr, kidx, kcnt, 0, softmax_scale, out_dtype, out, lse,
+                       ws, L, st);
+}

@@ -179,6 +179,31 @@ int masked_block_attn_fwd(bsva_shape s, const int8_t* q8, const float* q_scale,
                           size_t workspace_bytes,
                           bsva_stream_t stream);
 
+/* masked_block_attn_fwd without a workspace. The source pages have no
+ * counterpart: this entry point is for callers that cannot allocate device
+ * memory, such as a plugin inside a host application whose allocator already
+ * owns the device (on a small card every byte is budgeted, and a private
+ * cudaMalloc can fail or fragment the host's pool), or code on a streaming
+ * path that must not call cudaMalloc because it can synchronise the device.
+ * The kept-block lists live in a scratch array compiled into the library:
+ * 8,651,008 bytes on every GPU that loads it, held until the process exits.
+ * Limits: B*H*nQB <= 65,536 and B*H*nQB*nKB <= 2,097,152; a larger shape
+ * returns BSVA_ERR_WORKSPACE and launches nothing.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture. Every call shares the one array, which keeps the
+ * last call's contents: calls whose GPU work overlaps (two streams, two host
+ * threads) race on it, so the caller must serialise them. A device-side wait
+ * that runs out is recorded in the array's status word, which this entry
+ * point cannot report; use masked_block_attn_fwd and bsva_check_status where
+ * that matters. Other arguments as in masked_block_attn_fwd. */
+int masked_block_attn_fwd_noalloc(bsva_shape s, const int8_t* q8,
+                                  const float* q_scale, const int8_t* k8,
+                                  const float* k_scale, const void* v,
+                                  const uint8_t* block_mask, int mask_heads,
+                                  float softmax_scale, int out_dtype, void* out,
+                                  float* lse, bsva_stream_t stream);
+
 /* Synchronises `stream`, reads and clears the workspace's status word.
  * Returns BSVA_OK, or BSVA_ERR_DEVICE_TIMEOUT if a kernel's bounded wait gave
  * up since the last check (its outputs are then invalid). */
