@@ -11,9 +11,12 @@
 //              TMEM, scales, online max/sum, writes P (bf16) back to TMEM,
 //              rescales O in TMEM when the running max grows by more than
 //              2^8, and runs the epilogue O / l.
-//   warp 4     TMA producer: Q tile once, then K (int8) and V (bf16) tiles of
-//              the kept blocks, then the centroid tiles, NS-stage ring.
-//   warp 5     TMEM owner (alloc/dealloc) and single-thread MMA issuer:
+//   warp 4     TMA producer: Q tile once, then K (int8) tiles into a 4-stage
+//              ring (freed when QK is done) one tile ahead of V (bf16) tiles
+//              and per-tile metadata in a 3-stage ring (freed when PV is done):
+//              first the kept blocks, then the centroid tiles.
+//   warp 5     TMEM owner (alloc/dealloc) and single-thread MMA issuer (an
+//              event loop over the QK and PV queues):
 //              S = Q8 . K8^T with tcgen05.mma kind::i8 (M=128, N=64, int32
 //              accumulate) and O += P . V with kind::f16 (A = P from TMEM,
 //              B = V from shared memory, fp32 accumulate). S is double
@@ -30,19 +33,34 @@
 namespace bsva {
 namespace {
 
-constexpr int NS = 3;           // K/V pipeline stages
+constexpr int NK = 4;           // K tile stages (freed once QK of the tile is done)
+constexpr int NV = 3;           // V tile + metadata stages (freed once PV is done)
 constexpr int kThreads = 192;
 constexpr float kRescaleLog2 = 8.0f;   // lazy O rescale threshold (factor 256)
 constexpr uint32_t kTmemCols = 256;
 
+// Per-stage tile description, written by the producer warp before it arms
+// the stage's barrier and read by the softmax warps after QK of that tile.
+struct TileMeta {
+  float fac[32];    // centroid tiles: logit factor per group (sq*scale*log2e*sk/|g|)
+  float bias[32];   // centroid tiles: log2|g|, or -inf (kept block / no group)
+  float f;          // kept tiles: sq*sk*scale*log2e
+  int nvalid;       // kept tiles: valid key columns (64 except a tail block)
+  int centroid;     // 1 = centroid tile
+  int pad;
+};
+
 template <int D>
 struct __align__(1024) Smem {
   int8_t q[QB * D];
-  int8_t k[NS][KB * D];
-  __nv_bfloat16 v[NS][KB * D];
+  int8_t k[NK][KB * D];
+  __nv_bfloat16 v[NV][KB * D];
+  TileMeta meta[NV];
   uint64_t q_full;
-  uint64_t kv_full[NS];
-  uint64_t kv_empty[NS];
+  uint64_t k_full[NK];
+  uint64_t k_empty[NK];
+  uint64_t v_full[NV];
+  uint64_t v_empty[NV];
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t pv_done;
@@ -50,6 +68,12 @@ struct __align__(1024) Smem {
   uint32_t tmem_base;
   int abort;
 };
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float y;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+  return y;
+}
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -92,9 +116,13 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (tid == 0) {
     mbar_init(&sm.q_full, 1);
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&sm.kv_full[s], 1);
-      mbar_init(&sm.kv_empty[s], 1);
+    for (int s = 0; s < NK; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+    }
+    for (int s = 0; s < NV; ++s) {
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.s_full[b], 1);
@@ -118,36 +146,106 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
+    // One warp, two cursors: the K tile of step n+1 is issued before the V
+    // tile (and metadata) of step n, so K runs a tile ahead. Kept indices and
+    // their scales are fetched 32 tiles at a time, one per lane; centroid
+    // metadata is fetched a tile ahead, one group per lane. Lane 0 issues TMA.
+    const float sqs = a.q_scale[row_item] * a.scale_log2e;
+    const int32_t* kidx = a.kept_idx + row_item * a.nKB;
+    const uint8_t* kmask = a.kept_mask ? a.kept_mask + row_item * a.nKB : nullptr;
+    const float* cfac = a.cfac ? a.cfac + size_t(bh) * a.nCT * 32 : nullptr;
+    const float* cbias = a.cbias ? a.cbias + size_t(bh) * a.nCT * 32 : nullptr;
     if (lane == 0) {
       tma_prefetch_desc(&maps.q8);
       tma_prefetch_desc(&maps.k8);
       tma_prefetch_desc(&maps.v);
       mbar_arrive_expect_tx(&sm.q_full, QB * D);
       tma_load_3d(sm.q, &maps.q8, 0, q0, bh, &sm.q_full);
-      const int32_t* kidx = a.kept_idx + row_item * a.nKB;
-      for (int n = 0; n < N; ++n) {
-        const int s = n % NS;
-        if (n >= NS && !mbar_wait(&sm.kv_empty[s], ((n / NS) - 1) & 1, abort, a.status, lim)) break;
-        mbar_arrive_expect_tx(&sm.kv_full[s], KB * D * 3);
-        const CUtensorMap* mk;
-        const CUtensorMap* mv;
-        int row;
-        if (n < n_exact) {
-          row = kidx[n] * KB;
-          mk = &maps.k8;
-          mv = &maps.v;
-        } else {
-          row = (n - n_exact) * KB;
-          mk = &maps.ck8;
-          mv = &maps.cv;
+    }
+    int chunk_j = 0;          // kept index of tile (32*c + lane) of the current chunk
+    float chunk_f = 0.f;
+    int j_cur = 0, j_next = 0;   // key block of the V step's tile and of the K step's tile
+    float f_cur = 0.f, f_next = 0.f;
+    float cf_next = 0.f, cb_next = 0.f;   // centroid metadata of the next centroid tile
+    bool ok = true;
+
+    // group metadata of centroid tile t for this lane
+    auto cent_meta = [&](int t, float& fac, float& bias) {
+      const int G = t * 32 + lane;
+      const int jb = G / a.centroid_mode;
+      const bool kept = jb >= a.nKB || kmask[jb];
+      fac = sqs * cfac[G];
+      bias = kept ? -INFINITY : cbias[G];
+    };
+    auto k_step = [&](int t) -> bool {
+      const int sk = t % NK;
+      if (t >= NK && !__all_sync(0xffffffffu, mbar_wait(&sm.k_empty[sk], ((t / NK) - 1) & 1, abort, a.status, lim)))
+        return false;
+      int row;
+      if (t < n_exact) {
+        if ((t & 31) == 0) {
+          const int nn = t + lane;
+          chunk_j = nn < n_exact ? kidx[nn] : 0;
+          chunk_f = nn < n_exact ? sqs * a.k_scale[size_t(bh) * a.nKB + chunk_j] : 0.f;
         }
-        tma_load_3d(sm.k[s], mk, 0, row, bh, &sm.kv_full[s]);
-        tma_load_3d(sm.v[s], mv, 0, row, bh, &sm.kv_full[s]);
-        if (D == 128) tma_load_3d(sm.v[s] + KB * 64, mv, 64, row, bh, &sm.kv_full[s]);
+        j_next = __shfl_sync(0xffffffffu, chunk_j, t & 31);
+        f_next = __shfl_sync(0xffffffffu, chunk_f, t & 31);
+        row = j_next * KB;
+      } else {
+        row = (t - n_exact) * KB;
       }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&sm.k_full[sk], KB * D);
+        tma_load_3d(sm.k[sk], t < n_exact ? &maps.k8 : &maps.ck8, 0, row, bh, &sm.k_full[sk]);
+      }
+      return true;
+    };
+    auto v_step = [&](int t) -> bool {
+      const int sv = t % NV;
+      if (t >= NV && !__all_sync(0xffffffffu, mbar_wait(&sm.v_empty[sv], ((t / NV) - 1) & 1, abort, a.status, lim)))
+        return false;
+      TileMeta& mt = sm.meta[sv];
+      int row;
+      if (t < n_exact) {
+        row = j_cur * KB;
+        if (lane == 0) {
+          mt.f = f_cur;
+          mt.nvalid = min(KB, a.Lk - row);
+          mt.centroid = 0;
+        }
+      } else {
+        const int tc = t - n_exact;
+        row = tc * KB;
+        float fac, bias;
+        if (tc == 0) cent_meta(0, fac, bias);
+        else { fac = cf_next; bias = cb_next; }
+        mt.fac[lane] = fac;
+        mt.bias[lane] = bias;
+        if (lane == 0) mt.centroid = 1;
+        if (t + 1 < N) cent_meta(tc + 1, cf_next, cb_next);   // prefetch the next centroid tile
+      }
+      __syncwarp();
+      if (lane == 0) {
+        const CUtensorMap* mv = t < n_exact ? &maps.v : &maps.cv;
+        mbar_arrive_expect_tx(&sm.v_full[sv], KB * D * 2);
+        tma_load_3d(sm.v[sv], mv, 0, row, bh, &sm.v_full[sv]);
+        if (D == 128) tma_load_3d(sm.v[sv] + KB * 64, mv, 64, row, bh, &sm.v_full[sv]);
+      }
+      return true;
+    };
+
+    ok = k_step(0);
+    for (int n = 0; ok && n < N; ++n) {
+      j_cur = j_next;
+      f_cur = f_next;
+      if (n + 1 < N) ok = k_step(n + 1);
+      if (ok) ok = v_step(n);
     }
   } else if (warp == 5) {
     // ---------------------------------------------------------- MMA issuer
+    // Event loop: issue QK of the next tile when its K tile has landed (at most
+    // one tile ahead of PV: S is double buffered and P of tile n lives in S
+    // buffer n&1) and PV of the oldest pending tile once its P and V are ready.
     if (lane == 0) {
       // K-major INT8 tiles: rows of D bytes, 8-row groups of 8*D bytes.
       constexpr uint32_t kLayoutQK = (D == 128) ? 2u : 4u;   // 128B / 64B swizzle
@@ -160,38 +258,51 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint64_t dq = make_sdesc(smem_u32(sm.q), 16, kSboQK, kLayoutQK);
       bool ok = mbar_wait(&sm.q_full, 0, abort, a.status, lim);
       tc_fence_after();
-
-      auto issue_qk = [&](int n) -> bool {
-        const int s = n % NS;
-        if (!mbar_wait(&sm.kv_full[s], (n / NS) & 1, abort, a.status, lim)) return false;
-        tc_fence_after();
-        const uint64_t dk = make_sdesc(smem_u32(sm.k[s]), 16, kSboQK, kLayoutQK);
-        const uint32_t dS = tmem + ((n & 1) ? S_COL1 : S_COL0);
+      int nq = 0, np = 0;
+      uint64_t t_idle = 0;
+      while (ok && np < N) {
+        bool progressed = false;
+        if (nq < N && nq <= np + 1 && mbar_try_wait(&sm.k_full[nq % NK], (nq / NK) & 1)) {
+          tc_fence_after();
+          const int sk = nq % NK;
+          const uint64_t dk = make_sdesc(smem_u32(sm.k[sk]), 16, kSboQK, kLayoutQK);
+          const uint32_t dS = tmem + ((nq & 1) ? S_COL1 : S_COL0);
 #pragma unroll
-        for (int kk = 0; kk < D / 32; ++kk)   // K = 32 bytes per MMA
-          mma_i8_ss(dS, dq + 2 * kk, dk + 2 * kk, IDESC_QK, kk > 0 ? 1u : 0u);
-        tc_commit(&sm.s_full[n & 1]);
-        return true;
-      };
-      auto issue_pv = [&](int n) -> bool {
-        if (!mbar_wait(&sm.p_full[n & 1], (n >> 1) & 1, abort, a.status, lim)) return false;
-        tc_fence_after();
-        const int s = n % NS;
-        const uint64_t dv = make_sdesc(smem_u32(sm.v[s]), kLboV, kSboV, 2u);
-        const uint32_t aP = tmem + ((n & 1) ? S_COL1 : S_COL0);
+          for (int kk = 0; kk < D / 32; ++kk)   // K = 32 bytes per MMA
+            mma_i8_ss(dS, dq + 2 * kk, dk + 2 * kk, IDESC_QK, kk > 0 ? 1u : 0u);
+          tc_commit(&sm.k_empty[sk]);
+          tc_commit(&sm.s_full[nq & 1]);
+          ++nq;
+          progressed = true;
+        }
+        if (np < nq && mbar_try_wait(&sm.p_full[np & 1], (np >> 1) & 1) &&
+            mbar_try_wait(&sm.v_full[np % NV], (np / NV) & 1)) {
+          tc_fence_after();
+          const int sv = np % NV;
+          const uint64_t dv = make_sdesc(smem_u32(sm.v[sv]), kLboV, kSboV, 2u);
+          const uint32_t aP = tmem + ((np & 1) ? S_COL1 : S_COL0);
 #pragma unroll
-        for (int kk = 0; kk < KB / 16; ++kk)   // K = 16 keys per MMA: 8 TMEM columns of P, 16 rows of V
-          mma_bf16_ts(tmem + O_COL, aP + 8 * kk, dv + (16 * 128 / 16) * kk, IDESC_PV,
-                      (n > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&sm.kv_empty[s]);
-        tc_commit(&sm.pv_done);
-        return true;
-      };
-
-      if (ok) ok = issue_qk(0);
-      for (int n = 0; ok && n < N; ++n) {
-        if (n + 1 < N) ok = issue_qk(n + 1);
-        if (ok) ok = issue_pv(n);
+          for (int kk = 0; kk < KB / 16; ++kk)   // K = 16 keys per MMA: 8 TMEM columns of P, 16 rows of V
+            mma_bf16_ts(tmem + O_COL, aP + 8 * kk, dv + (16 * 128 / 16) * kk, IDESC_PV,
+                        (np > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(&sm.v_empty[sv]);
+          tc_commit(&sm.pv_done);
+          ++np;
+          progressed = true;
+        }
+        if (progressed) {
+          t_idle = 0;
+        } else {
+          if (*abort) break;
+          const uint64_t now = globaltimer_ns();
+          if (t_idle == 0) {
+            t_idle = now;
+          } else if (now - t_idle > lim) {
+            *abort = 1;
+            atomicOr(a.status, kStatusTimeout);
+            break;
+          }
+        }
       }
       tc_commit(&sm.o_full);
     }
@@ -199,117 +310,153 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ------------------------------------------------------------- softmax
     const int r = tid;                                   // row within the block
     const uint32_t lane_base = uint32_t(warp * 32) << 16;
-    const float sqs = a.q_scale[row_item] * a.scale_log2e;
-    const int32_t* kidx = a.kept_idx + row_item * a.nKB;
-    const uint8_t* kmask = a.kept_mask ? a.kept_mask + row_item * a.nKB : nullptr;
-    const float* cfac = a.cfac + size_t(bh) * a.nCT * 32;
-    const float* cbias = a.cbias + size_t(bh) * a.nCT * 32;
+    const bool want_lse = a.lse != nullptr;
     float m_ref = -INFINITY, l = 0.f, le = 0.f;
     bool alive = true;
+    int n_cur = 0;
+    // O *= alpha in TMEM once the PV product of the previous tile has landed.
+    auto rescale_o = [&](float alpha) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done, (n_cur - 1) & 1, abort, a.status, lim))) return false;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_base + O_COL + c0, o);
+        tmem_wait_ld(o);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+        tmem_st32(tmem + lane_base + O_COL + c0, o);
+      }
+      tmem_wait_st();
+      return true;
+    };
 
     for (int n = 0; n < N; ++n) {
-      const bool exact = n < n_exact;
-      float f = 0.f;
-      int nvalid = 0;
-      float gf[32], gb[32];
-      if (exact) {
-        const int j = kidx[n];
-        f = sqs * a.k_scale[size_t(bh) * a.nKB + j];
-        nvalid = min(KB, a.Lk - j * KB);
-      } else {
-        const int t = n - n_exact;
-        const float4* fp = reinterpret_cast<const float4*>(cfac + t * 32);
-        const float4* bp = reinterpret_cast<const float4*>(cbias + t * 32);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 fv = fp[q], bv = bp[q];
-          gf[4 * q] = fv.x; gf[4 * q + 1] = fv.y; gf[4 * q + 2] = fv.z; gf[4 * q + 3] = fv.w;
-          gb[4 * q] = bv.x; gb[4 * q + 1] = bv.y; gb[4 * q + 2] = bv.z; gb[4 * q + 3] = bv.w;
-        }
-#pragma unroll
-        for (int g = 0; g < 32; ++g) {
-          const int jb = (t * 32 + g) / a.centroid_mode;
-          const bool kept = jb < a.nKB && kmask[jb];
-          gf[g] *= sqs;
-          if (kept) gb[g] = -INFINITY;
-        }
-      }
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[n & 1], (n >> 1) & 1, abort, a.status, lim))) {
+      n_cur = n;
+      const int s = n % NV;
+      bool ok = mbar_wait(&sm.s_full[n & 1], (n >> 1) & 1, abort, a.status, lim);
+      // the tile's metadata is published with its V stage's barrier
+      ok = ok && mbar_wait(&sm.v_full[s], (n / NV) & 1, abort, a.status, lim);
+      if (!__all_sync(0xffffffffu, ok)) {
         alive = false;
         break;
       }
       tc_fence_after();
+      const TileMeta& mt = sm.meta[s];
+      const bool cent = mt.centroid != 0;
       const uint32_t sc = (n & 1) ? S_COL1 : S_COL0;
-      uint32_t sr[64];
-      tmem_ld64(tmem + lane_base + sc, sr);
-      tmem_wait_ld();
+      uint32_t pk[32];
+      float lsum = 0.f, esum = 0.f;
 
-      float x[64];
-      float mt = -INFINITY;
-      if (exact) {
+      if (!cent) {
+        // ---- kept tile: logits x = S * f (log2 units), 64 keys per row.
+        // f = 0 (an all-zero Q or K block) would turn a masked -inf into NaN;
+        // 1e-30 keeps every valid logit within 1e-23 of 0 and masked ones at -inf.
+        const float f = fmaxf(mt.f, 1e-30f);
+        const int nvalid = mt.nvalid;
+        float xs[64];
+        uint32_t sa[32], sb[32];
+        tmem_ld32(tmem + lane_base + sc, sa);
+        tmem_wait_ld(sa);
+        tmem_ld32(tmem + lane_base + sc + 32, sb);    // in flight while the first half converts
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          x[c] = (c < nvalid) ? float(int(sr[c])) * f : -INFINITY;
-          mt = fmaxf(mt, x[c]);
-        }
-      } else {
+        for (int c = 0; c < 32; ++c) xs[c] = float(int(sa[c]));
+        tmem_wait_ld(sb);
 #pragma unroll
-        for (int g = 0; g < 32; ++g) {
-          const int dot = 128 * int(sr[2 * g]) + int(sr[2 * g + 1]);
-          x[g] = (gb[g] == -INFINITY) ? -INFINITY : fmaf(float(dot), gf[g], gb[g]);
-          mt = fmaxf(mt, x[g]);
+        for (int c = 0; c < 32; ++c) xs[32 + c] = float(int(sb[c]));
+        if (nvalid < KB) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c >= nvalid) xs[c] = -INFINITY;
         }
-      }
-
-      // lazy rescale: only when the running max grows by more than 2^8
-      const bool need = mt > m_ref + kRescaleLog2;
-      if (__any_sync(0xffffffffu, need)) {
-        const float m_new = need ? mt : m_ref;
-        const float alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new);
-        if (n > 0) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done, (n - 1) & 1, abort, a.status, lim))) {
+        // P = 2^(x*f - m) as bf16 pairs; lsum adds the bf16-rounded weights
+        // the PV product uses, esum the unrounded ones (log-sum-exp only).
+        auto exps = [&](float m_use) {
+          const float2 f2 = make_float2(f, f), nm2 = make_float2(-m_use, -m_use);
+          float2 la = make_float2(0.f, 0.f), ea = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float2 y = __ffma2_rn(make_float2(xs[2 * c], xs[2 * c + 1]), f2, nm2);
+            const float p0 = ex2(y.x), p1 = ex2(y.y);
+            pk[c] = pack_bf16x2(p0, p1);
+            la = __fadd2_rn(la, make_float2(__uint_as_float(pk[c] << 16), __uint_as_float(pk[c] & 0xFFFF0000u)));
+            if (want_lse) ea = __fadd2_rn(ea, make_float2(p0, p1));
+          }
+          lsum = la.x + la.y;
+          esum = ea.x + ea.y;
+        };
+        // Speculate that the running max still holds (it nearly always does
+        // after the first tiles), so the exps need not wait for this tile's max.
+        const bool first = __all_sync(0xffffffffu, m_ref == -INFINITY);
+        if (!first) exps(m_ref);
+        float m8[22];
+#pragma unroll
+        for (int c = 0; c < 21; ++c) m8[c] = fmax3(xs[3 * c], xs[3 * c + 1], xs[3 * c + 2]);
+        m8[21] = xs[63];
+#pragma unroll
+        for (int c = 0; c < 7; ++c) m8[c] = fmax3(m8[3 * c], m8[3 * c + 1], m8[3 * c + 2]);
+        m8[0] = fmax3(m8[0], m8[1], m8[2]);
+        m8[1] = fmax3(m8[3], m8[4], m8[5]);
+        m8[2] = fmax3(m8[6], m8[21], m8[0]);
+        const float mt_max = fmaxf(m8[1], m8[2]) * f;   // f > 0: the max commutes with the scale
+        const bool need = mt_max > m_ref + kRescaleLog2;
+        if (first || __any_sync(0xffffffffu, need)) {
+          const float m_new = need ? mt_max : m_ref;
+          const float alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new);
+          if (n > 0 && !rescale_o(alpha)) {
             alive = false;
             break;
           }
-          tc_fence_after();
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(tmem + lane_base + O_COL + c0, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(tmem + lane_base + O_COL + c0, o);
-          }
-          tmem_wait_st();
-        }
-        l *= alpha;
-        le *= alpha;
-        m_ref = m_new;
-      }
-      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-
-      uint32_t pk[32];
-      float lsum = 0.f;
-      // Two row sums: lb adds the bf16-rounded weights that the PV product uses
-      // (numerator and denominator then see the same probabilities), le adds
-      // the unrounded weights for the log-sum-exp.
-      float esum = 0.f;
-      if (exact) {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float p0 = ex2(x[2 * c] - m_use), p1 = ex2(x[2 * c + 1] - m_use);
-          pk[c] = pack_bf16x2(p0, p1);
-          lsum += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xFFFF0000u);
-          esum += p0 + p1;
+          l *= alpha;
+          le *= alpha;
+          m_ref = m_new;
+          exps(m_ref == -INFINITY ? 0.f : m_ref);
         }
       } else {
+        // ---- centroid tile: 32 groups, each an exact int dot from its (hi, lo) rows
+        uint32_t sa[32], sb[32];
+        tmem_ld32(tmem + lane_base + sc, sa);
+        tmem_wait_ld(sa);
+        tmem_ld32(tmem + lane_base + sc + 32, sb);
+        float xs[32];
+#pragma unroll
+        for (int g = 0; g < 16; ++g) {
+          const int dot = 128 * int(sa[2 * g]) + int(sa[2 * g + 1]);
+          xs[g] = fmaf(float(dot), mt.fac[g], mt.bias[g]);   // bias -inf masks the group
+        }
+        tmem_wait_ld(sb);
+#pragma unroll
+        for (int g = 0; g < 16; ++g) {
+          const int dot = 128 * int(sb[2 * g]) + int(sb[2 * g + 1]);
+          xs[16 + g] = fmaf(float(dot), mt.fac[16 + g], mt.bias[16 + g]);
+        }
+        float m8[11];
+#pragma unroll
+        for (int c = 0; c < 10; ++c) m8[c] = fmax3(xs[3 * c], xs[3 * c + 1], xs[3 * c + 2]);
+        m8[10] = fmaxf(xs[30], xs[31]);
+        m8[0] = fmax3(m8[0], m8[1], m8[2]);
+        m8[1] = fmax3(m8[3], m8[4], m8[5]);
+        m8[2] = fmax3(m8[6], m8[7], m8[8]);
+        const float mt_max = fmax3(fmax3(m8[0], m8[1], m8[2]), m8[9], m8[10]);
+        const bool need = mt_max > m_ref + kRescaleLog2;
+        if (__any_sync(0xffffffffu, need)) {
+          const float m_new = need ? mt_max : m_ref;
+          const float alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new);
+          if (n > 0 && !rescale_o(alpha)) {
+            alive = false;
+            break;
+          }
+          l *= alpha;
+          le *= alpha;
+          m_ref = m_new;
+        }
+        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
 #pragma unroll
         for (int g = 0; g < 32; ++g) {
-          const float p = ex2(x[g] - m_use);
+          const float p = ex2(xs[g] - m_use);
           pk[g] = pack_bf16x2(p, p);
           lsum += __uint_as_float(pk[g] << 16);
-          esum += p;
+          if (want_lse) esum += p;
         }
       }
       l += lsum;
