@@ -130,7 +130,8 @@ def _dist():
 def _max_over_ranks(dist, x: float) -> float:
     if dist is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -138,7 +139,8 @@ def _max_over_ranks(dist, x: float) -> float:
 def _barrier(dist):
     if dist is not None:
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def kept_work(route, w):
@@ -234,6 +236,33 @@ def run_steps(st: SolStep, steps: int, warmup: int, dist, sampler=None):
                 centroid_ms=_max_over_ranks(dist, t_cent), attn_ms=_max_over_ranks(dist, t_attn)), clocks
 
 
+ATTN_SOURCES = ("block_sparse_video_int8_b200/csrc/attn_sm100.cu", "block_sparse_video_int8_b200/csrc/common.cuh")
+TRAFFIC_FILE = "profiles/attn_sm100_traffic.md"
+
+
+def attn_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ATTN_SOURCES:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary, or None
+    if there is none for this workload or the kernel changed since it was taken."""
+    path = os.path.join(ROOT, TRAFFIC_FILE)
+    if not os.path.exists(path):
+        return None
+    src, val = None, None
+    for line in open(path):
+        if line.startswith("kernel_sources_sha256:"):
+            src = line.split(":", 1)[1].strip()
+        if line.startswith(f"dram_bytes_per_launch[{workload}]:"):
+            val = int(line.split(":", 1)[1].strip())
+    return val if (src == attn_source_hash() and val is not None) else None
+
+
 def roofline_numbers(w, work, r, peaks):
     p_bf16 = peaks["bf16"] * 1e12
     p_int8 = 2.0 * p_bf16                       # nominal dense INT8 : bf16 ratio on B200
@@ -245,7 +274,7 @@ def roofline_numbers(w, work, r, peaks):
     rb = route_bytes(w)
     return dict(
         attn=dict(bound="tensor", achieved=round(achieved, 2), peak=round(peak_eff, 2), unit="TFLOP/s",
-                  frac=round(achieved / peak_eff, 4), traffic=None),
+                  frac=round(achieved / peak_eff, 4), traffic=measured_traffic(w.name)),
         route=dict(bound="hbm", achieved=round(rb / (r["route_ms"] * 1e-3) / 1e9, 1), peak=peaks["hbm"],
                    unit="GB/s", frac=round(rb / (r["route_ms"] * 1e-3) / 1e9 / peaks["hbm"], 4),
                    bytes=rb),
@@ -443,7 +472,7 @@ def main():
         e2e = e2e_measure(bsva, w, args.tau, Qp, Kp, Vp, max(3, args.steps // 10), 2, dist)
     cpu = None
     if rank == 0 and world == 1 and not args.quick:
-        v_ms, sample, secs = oracle_sample(w, args.tau, 2, 24)
+        v_ms, sample, secs = oracle_sample(w, args.tau, 4, 384)
         cpu = {"value": round(v_ms, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": sample + f" ({secs:.1f} s of CPU work)"}
 
