@@ -43,7 +43,7 @@ import workloads  # noqa: E402
 
 METRIC = "sparse-attn ms/call + dense-equiv TFLOPS at Wan-14B-like shape; % of roofline"
 UNIT = "ms/call"
-LAUNCHES_PER_STEP = 4          # quant_pool, route, centroids, attention
+LAUNCHES_PER_STEP = 5          # quant_pool, score, select, centroids, attention
 
 
 def _peaks():
@@ -183,7 +183,8 @@ class SolStep:
         self.bsva, self.w, self.tau = bsva, w, tau
         self.Q, self.K, self.V = Q, K, V
         self.route = bsva.sparse_attn_route(Q, K, tau, n_prefix=w.n_prefix)
-        self.ws = bsva.new_workspace(self.route.shape, w.centroid_mode)
+        self.ws = bsva.new_workspace(self.route.shape, w.centroid_mode)   # also serves routing
+        self.route.scratch = None
         self.out = torch.empty_like(Q)
         self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
         self.t_route = self.t_cent = self.t_attn = 0.0
@@ -192,7 +193,7 @@ class SolStep:
     def step(self, timed=True):
         b, w, ev = self.bsva, self.w, self.ev
         ev[0].record()
-        b.sparse_attn_route(self.Q, self.K, self.tau, n_prefix=w.n_prefix, out=self.route)
+        b.sparse_attn_route(self.Q, self.K, self.tau, n_prefix=w.n_prefix, out=self.route, workspace=self.ws)
         ev[1].record()
         b.build_centroids(self.route, self.V, w.centroid_mode, self.ws)
         ev[2].record()
@@ -299,7 +300,7 @@ def e2e_measure(bsva, w, tau, Qh, Kh, Vh, steps, warmup, dist):
         Q.copy_(Qh, non_blocking=True)
         K.copy_(Kh, non_blocking=True)
         V.copy_(Vh, non_blocking=True)
-        route = bsva.sparse_attn_route(Q, K, tau, n_prefix=w.n_prefix, out=route)
+        route = bsva.sparse_attn_route(Q, K, tau, n_prefix=w.n_prefix, out=route, workspace=ws)
         if ws is None:
             ws = bsva.new_workspace(route.shape, w.centroid_mode)
         out = bsva.sparse_attn_fwd(route, V, w.centroid_mode, workspace=ws, out=out)

@@ -22,12 +22,12 @@ import torch
 
 __all__ = [
     "BsvaError", "load", "lib_path", "Route", "Shape", "abi_version",
-    "workspace_bytes", "quantize_qk", "sparse_attn_route", "sparse_attn_fwd",
+    "workspace_bytes", "route_workspace_bytes", "quantize_qk", "sparse_attn_route", "sparse_attn_fwd",
     "masked_block_attn_fwd", "check_status", "selftest_timeout", "new_workspace",
     "build_centroids", "sparse_attn_core",
 ]
 
-ABI_VERSION = 1
+ABI_VERSION = 2
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
 
@@ -58,8 +58,9 @@ _SIGS = {
     "bsva_last_error": (ctypes.c_char_p, []),
     "bsva_workspace_bytes": (ctypes.c_size_t, [Shape, ctypes.c_int]),
     "bsva_quantize_qk": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "bsva_route_workspace_bytes": (ctypes.c_size_t, [Shape]),
     "sparse_attn_route": (ctypes.c_int, [Shape, _P, _P, ctypes.c_double, _P, _P, _P, _P, _P, _P,
-                                         _P, _P, _P, _P, _P]),
+                                         _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "sparse_attn_fwd": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int,
                                        ctypes.c_float, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
     "masked_block_attn_fwd": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, _P, ctypes.c_int,
@@ -169,6 +170,7 @@ class Route:
     kept_idx: torch.Tensor
     kept_cnt: torch.Tensor
     row_stats: torch.Tensor | None
+    scratch: torch.Tensor | None = None   # route-only workspace when the caller passes none
 
 
 def _alloc_quant(s: Shape, dev):
@@ -196,9 +198,21 @@ def quantize_qk(q: torch.Tensor, k: torch.Tensor, out: dict | None = None, strea
     return o
 
 
+def route_workspace_bytes(shape: Shape) -> int:
+    n = load().bsva_route_workspace_bytes(shape)
+    if n == 0:
+        raise BsvaError(1, f"bad shape for a routing workspace: {_fmt(shape)}")
+    return n
+
+
 def sparse_attn_route(q: torch.Tensor, k: torch.Tensor, tau: float, n_prefix: int = 0,
-                      row_stats: bool = False, out: Route | None = None, stream=None) -> Route:
-    """Quantise, score and route (C ABI ``sparse_attn_route``)."""
+                      row_stats: bool = False, out: Route | None = None,
+                      workspace: torch.Tensor | None = None, stream=None) -> Route:
+    """Quantise, score and route (C ABI ``sparse_attn_route``).
+
+    ``workspace`` is a device uint8 buffer of at least ``route_workspace_bytes``
+    (a ``new_workspace`` buffer serves too); without one, a route-only buffer is
+    allocated once and kept on the returned ``Route``."""
     lib = load()
     s = _shape_of(q, k, n_prefix)
     _need(q, torch.bfloat16, None, "q")
@@ -215,10 +229,18 @@ def sparse_attn_route(q: torch.Tensor, k: torch.Tensor, tau: float, n_prefix: in
                                if row_stats else None))
     else:
         out.shape, out.tau = s, tau
+    if workspace is None:
+        need = lib.bsva_route_workspace_bytes(s)   # 0 on a bad shape: the call below reports it
+        if need and (out.scratch is None or out.scratch.numel() < need):
+            out.scratch = torch.empty(need, dtype=torch.uint8, device=q.device)
+        workspace = out.scratch
+    if workspace is not None:
+        _need(workspace, torch.uint8, None, "workspace")
     _check(lib.sparse_attn_route(s, _ptr(q), _ptr(k), ctypes.c_double(tau), _ptr(out.q8),
                                  _ptr(out.q_scale), _ptr(out.k8), _ptr(out.k_scale), _ptr(out.q_pool),
                                  _ptr(out.k_pool), _ptr(out.kept_mask), _ptr(out.kept_idx),
-                                 _ptr(out.kept_cnt), _ptr(out.row_stats), _stream(stream)))
+                                 _ptr(out.kept_cnt), _ptr(out.row_stats), _ptr(workspace),
+                                 0 if workspace is None else workspace.numel(), _stream(stream)))
     return out
 
 

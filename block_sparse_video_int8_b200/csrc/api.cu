@@ -15,7 +15,6 @@
 #include "common.cuh"
 
 namespace bsva {
-bool route_supported(int nKB, int d);
 }
 
 using namespace bsva;
@@ -184,6 +183,11 @@ size_t bsva_workspace_bytes(bsva_shape s, int centroid_mode) {
   return ws_layout(s, centroid_mode).total;
 }
 
+size_t bsva_route_workspace_bytes(bsva_shape s) {
+  if (check_shape(s) != BSVA_OK) return 0;
+  return ws_layout(s, 1).route_total;
+}
+
 int bsva_quantize_qk(bsva_shape s, const void* q, const void* k, int8_t* q8, float* q_scale, int8_t* k8,
                      float* k_scale, int32_t* q_pool, int32_t* k_pool, bsva_stream_t stream) {
   int rc;
@@ -200,7 +204,8 @@ int bsva_quantize_qk(bsva_shape s, const void* q, const void* k, int8_t* q8, flo
 
 int sparse_attn_route(bsva_shape s, const void* q, const void* k, double tau, int8_t* q8, float* q_scale, int8_t* k8,
                       float* k_scale, int32_t* q_pool, int32_t* k_pool, uint8_t* kept_mask, int32_t* kept_idx,
-                      int32_t* kept_cnt, double* row_stats, bsva_stream_t stream) {
+                      int32_t* kept_cnt, double* row_stats, void* workspace, size_t workspace_bytes,
+                      bsva_stream_t stream) {
   int rc;
   if ((rc = check_shape(s))) return rc;
   if (std::isnan(tau)) return fail(BSVA_ERR_INVALID_ARG, "tau is NaN");
@@ -209,16 +214,16 @@ int sparse_attn_route(bsva_shape s, const void* q, const void* k, double tau, in
   REQUIRE_PTR(q_scale, 4); REQUIRE_PTR(k_scale, 4); REQUIRE_PTR(q_pool, 16); REQUIRE_PTR(k_pool, 16);
   REQUIRE_PTR(kept_mask, 1); REQUIRE_PTR(kept_idx, 4); REQUIRE_PTR(kept_cnt, 4);
   if (row_stats && !aligned(row_stats, 8)) return fail(BSVA_ERR_INVALID_ARG, "row_stats is not 8-byte aligned");
-  const int nKB = (s.Lk + KB - 1) / KB;
-  if (!route_supported(nKB, s.d))
-    return fail(BSVA_ERR_UNSUPPORTED, "Lk = %d: a routing row does not fit shared memory", s.Lk);
+  const WsLayout ws = ws_layout(s, 1);
+  if ((rc = check_workspace(workspace, workspace_bytes, ws.route_total))) return rc;
   if ((rc = check_device())) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  double* scores = reinterpret_cast<double*>(static_cast<unsigned char*>(workspace) + ws.scores);
   cudaError_t e = launch_quant_pool(s, reinterpret_cast<const __nv_bfloat16*>(q),
                                     reinterpret_cast<const __nv_bfloat16*>(k), q8, q_scale, k8, k_scale, q_pool,
                                     k_pool, st);
   if (e != cudaSuccess) return cuda_fail(e, "quant_pool launch");
-  e = launch_route(s, tau, q_pool, k_pool, k_scale, kept_mask, kept_idx, kept_cnt, row_stats, st);
+  e = launch_route(s, tau, q_pool, k_pool, k_scale, scores, kept_mask, kept_idx, kept_cnt, row_stats, st);
   if (e != cudaSuccess) return cuda_fail(e, "route launch");
   return ok();
 }

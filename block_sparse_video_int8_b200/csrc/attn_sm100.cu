@@ -11,12 +11,13 @@
 //              TMEM, scales, online max/sum, writes P (bf16) back to TMEM,
 //              rescales O in TMEM when the running max grows by more than
 //              2^8, and runs the epilogue O / l.
-//   warp 4     TMA producer: Q tile once, then K (int8) tiles into a 4-stage
-//              ring (freed when QK is done) one tile ahead of V (bf16) tiles
-//              and per-tile metadata in a 3-stage ring (freed when PV is done):
-//              first the kept blocks, then the centroid tiles.
-//   warp 5     TMEM owner (alloc/dealloc) and single-thread MMA issuer (an
-//              event loop over the QK and PV queues):
+//   warp 4     TMA producer: Q tile once, then K (int8) tiles with their
+//              per-tile metadata into a 4-stage ring (freed by the softmax
+//              warps once they are done with the tile) one tile ahead of V
+//              (bf16) tiles in a 3-stage ring (freed when PV is done): first
+//              the kept blocks, then the centroid tiles.
+//   warp 5     TMEM owner (alloc/dealloc) and MMA issuer (the warp runs the
+//              schedule, one elected lane issues):
 //              S = Q8 . K8^T with tcgen05.mma kind::i8 (M=128, N=64, int32
 //              accumulate) and O += P . V with kind::f16 (A = P from TMEM,
 //              B = V from shared memory, fp32 accumulate). S is double
@@ -33,14 +34,14 @@
 namespace bsva {
 namespace {
 
-constexpr int NK = 4;           // K tile stages (freed once QK of the tile is done)
-constexpr int NV = 3;           // V tile + metadata stages (freed once PV is done)
+constexpr int NK = 4;           // K tile + metadata stages (freed once the softmax is done with the tile)
+constexpr int NV = 3;           // V tile stages (freed once PV is done)
 constexpr int kThreads = 192;
 constexpr float kRescaleLog2 = 8.0f;   // lazy O rescale threshold (factor 256)
 constexpr uint32_t kTmemCols = 256;
 
 // Per-stage tile description, written by the producer warp before it arms
-// the stage's barrier and read by the softmax warps after QK of that tile.
+// the K stage's barrier and read by the softmax warps after QK of that tile.
 struct TileMeta {
   float fac[32];    // centroid tiles: logit factor per group (sq*scale*log2e*sk/|g|)
   float bias[32];   // centroid tiles: log2|g|, or -inf (kept block / no group)
@@ -55,7 +56,7 @@ struct __align__(1024) Smem {
   int8_t q[QB * D];
   int8_t k[NK][KB * D];
   __nv_bfloat16 v[NV][KB * D];
-  TileMeta meta[NV];
+  TileMeta meta[NK];
   uint64_t q_full;
   uint64_t k_full[NK];
   uint64_t k_empty[NK];
@@ -63,7 +64,6 @@ struct __align__(1024) Smem {
   uint64_t v_empty[NV];
   uint64_t s_full[2];
   uint64_t p_full[2];
-  uint64_t pv_done;
   uint64_t o_full;
   uint32_t tmem_base;
   int abort;
@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     mbar_init(&sm.q_full, 1);
     for (int s = 0; s < NK; ++s) {
       mbar_init(&sm.k_full[s], 1);
-      mbar_init(&sm.k_empty[s], 1);
+      mbar_init(&sm.k_empty[s], 4);   // released by the 4 softmax warps
     }
     for (int s = 0; s < NV; ++s) {
       mbar_init(&sm.v_full[s], 1);
@@ -128,7 +128,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&sm.s_full[b], 1);
       mbar_init(&sm.p_full[b], QB);
     }
-    mbar_init(&sm.pv_done, 1);
     mbar_init(&sm.o_full, 1);
     sm.abort = 0;
     fence_mbar_init();
@@ -146,8 +145,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
-    // One warp, two cursors: the K tile of step n+1 is issued before the V
-    // tile (and metadata) of step n, so K runs a tile ahead. Kept indices and
+    // One warp, two cursors: the K tile (and metadata) of step n+1 is issued
+    // before the V tile of step n, so K runs a tile ahead. Kept indices and
     // their scales are fetched 32 tiles at a time, one per lane; centroid
     // metadata is fetched a tile ahead, one group per lane. Lane 0 issues TMA.
     const float sqs = a.q_scale[row_item] * a.scale_log2e;
@@ -165,7 +164,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     int chunk_j = 0;          // kept index of tile (32*c + lane) of the current chunk
     float chunk_f = 0.f;
     int j_cur = 0, j_next = 0;   // key block of the V step's tile and of the K step's tile
-    float f_cur = 0.f, f_next = 0.f;
     float cf_next = 0.f, cb_next = 0.f;   // centroid metadata of the next centroid tile
     bool ok = true;
 
@@ -181,6 +179,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int sk = t % NK;
       if (t >= NK && !__all_sync(0xffffffffu, mbar_wait(&sm.k_empty[sk], ((t / NK) - 1) & 1, abort, a.status, lim)))
         return false;
+      TileMeta& mt = sm.meta[sk];
       int row;
       if (t < n_exact) {
         if ((t & 31) == 0) {
@@ -189,27 +188,10 @@ __global__ void __launch_bounds__(kThreads, 2)
           chunk_f = nn < n_exact ? sqs * a.k_scale[size_t(bh) * a.nKB + chunk_j] : 0.f;
         }
         j_next = __shfl_sync(0xffffffffu, chunk_j, t & 31);
-        f_next = __shfl_sync(0xffffffffu, chunk_f, t & 31);
+        const float f_next = __shfl_sync(0xffffffffu, chunk_f, t & 31);
         row = j_next * KB;
-      } else {
-        row = (t - n_exact) * KB;
-      }
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&sm.k_full[sk], KB * D);
-        tma_load_3d(sm.k[sk], t < n_exact ? &maps.k8 : &maps.ck8, 0, row, bh, &sm.k_full[sk]);
-      }
-      return true;
-    };
-    auto v_step = [&](int t) -> bool {
-      const int sv = t % NV;
-      if (t >= NV && !__all_sync(0xffffffffu, mbar_wait(&sm.v_empty[sv], ((t / NV) - 1) & 1, abort, a.status, lim)))
-        return false;
-      TileMeta& mt = sm.meta[sv];
-      int row;
-      if (t < n_exact) {
-        row = j_cur * KB;
         if (lane == 0) {
-          mt.f = f_cur;
+          mt.f = f_next;
           mt.nvalid = min(KB, a.Lk - row);
           mt.centroid = 0;
         }
@@ -224,7 +206,18 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (lane == 0) mt.centroid = 1;
         if (t + 1 < N) cent_meta(tc + 1, cf_next, cb_next);   // prefetch the next centroid tile
       }
-      __syncwarp();
+      __syncwarp();   // the metadata is published by lane 0's arrive on the stage's barrier
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&sm.k_full[sk], KB * D);
+        tma_load_3d(sm.k[sk], t < n_exact ? &maps.k8 : &maps.ck8, 0, row, bh, &sm.k_full[sk]);
+      }
+      return true;
+    };
+    auto v_step = [&](int t) -> bool {
+      const int sv = t % NV;
+      if (t >= NV && !__all_sync(0xffffffffu, mbar_wait(&sm.v_empty[sv], ((t / NV) - 1) & 1, abort, a.status, lim)))
+        return false;
+      const int row = t < n_exact ? j_cur * KB : (t - n_exact) * KB;
       if (lane == 0) {
         const CUtensorMap* mv = t < n_exact ? &maps.v : &maps.cv;
         mbar_arrive_expect_tx(&sm.v_full[sv], KB * D * 2);
@@ -237,75 +230,75 @@ __global__ void __launch_bounds__(kThreads, 2)
     ok = k_step(0);
     for (int n = 0; ok && n < N; ++n) {
       j_cur = j_next;
-      f_cur = f_next;
       if (n + 1 < N) ok = k_step(n + 1);
       if (ok) ok = v_step(n);
     }
   } else if (warp == 5) {
     // ---------------------------------------------------------- MMA issuer
-    // Event loop: issue QK of the next tile when its K tile has landed (at most
-    // one tile ahead of PV: S is double buffered and P of tile n lives in S
-    // buffer n&1) and PV of the oldest pending tile once its P and V are ready.
-    if (lane == 0) {
-      // K-major INT8 tiles: rows of D bytes, 8-row groups of 8*D bytes.
-      constexpr uint32_t kLayoutQK = (D == 128) ? 2u : 4u;   // 128B / 64B swizzle
-      constexpr uint32_t kSboQK = 8 * D;
-      // V tiles, MN-major bf16: 128-byte rows (64 d-values), 8-row groups of
-      // 1 KB, the two 64-column halves (D = 128) 8 KB apart.
-      constexpr uint32_t kLboV = KB * 128, kSboV = 1024;
-      constexpr uint32_t IDESC_QK = make_idesc(2, 1, 1, false, false, 128, 64);
-      constexpr uint32_t IDESC_PV = make_idesc(1, 1, 1, false, true, 128, D);
-      const uint64_t dq = make_sdesc(smem_u32(sm.q), 16, kSboQK, kLayoutQK);
-      bool ok = mbar_wait(&sm.q_full, 0, abort, a.status, lim);
-      tc_fence_after();
-      int nq = 0, np = 0;
-      uint64_t t_idle = 0;
-      while (ok && np < N) {
-        bool progressed = false;
-        if (nq < N && nq <= np + 1 && mbar_try_wait(&sm.k_full[nq % NK], (nq / NK) & 1)) {
-          tc_fence_after();
-          const int sk = nq % NK;
-          const uint64_t dk = make_sdesc(smem_u32(sm.k[sk]), 16, kSboQK, kLayoutQK);
-          const uint32_t dS = tmem + ((nq & 1) ? S_COL1 : S_COL0);
+    // K-major INT8 tiles: rows of D bytes, 8-row groups of 8*D bytes.
+    constexpr uint32_t kLayoutQK = (D == 128) ? 2u : 4u;   // 128B / 64B swizzle
+    constexpr uint32_t kSboQK = 8 * D;
+    // V tiles, MN-major bf16: 128-byte rows (64 d-values), 8-row groups of
+    // 1 KB, the two 64-column halves (D = 128) 8 KB apart.
+    constexpr uint32_t kLboV = KB * 128, kSboV = 1024;
+    constexpr uint32_t IDESC_QK = make_idesc(2, 1, 1, false, false, 128, 64);
+    constexpr uint32_t IDESC_PV = make_idesc(1, 1, 1, false, true, 128, D);
+    constexpr uint32_t kStrideK = (KB * D) >> 4, kStrideV = (KB * D * 2) >> 4;   // stage strides, 16 B units
+    const uint64_t dq = make_sdesc(smem_u32(sm.q), 16, kSboQK, kLayoutQK);
+    const uint64_t dk0 = make_sdesc(smem_u32(sm.k[0]), 16, kSboQK, kLayoutQK);
+    const uint64_t dv0 = make_sdesc(smem_u32(sm.v[0]), kLboV, kSboV, 2u);
+    // The whole warp runs the schedule (all values warp-uniform); one elected
+    // lane issues each group of MMAs and its commit (whole-warp issue with
+    // elect.sync measured faster than a single issuing thread).
+    // QK(n) into S buffer n&1: int8, K = 32 per MMA.
+    auto do_qk = [&](int n) {
+      const int sk = n % NK;
+      const uint64_t dk = dk0 + uint64_t(sk * kStrideK);
+      const uint32_t dS = tmem + ((n & 1) ? S_COL1 : S_COL0);
+      if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < D / 32; ++kk)   // K = 32 bytes per MMA
-            mma_i8_ss(dS, dq + 2 * kk, dk + 2 * kk, IDESC_QK, kk > 0 ? 1u : 0u);
-          tc_commit(&sm.k_empty[sk]);
-          tc_commit(&sm.s_full[nq & 1]);
-          ++nq;
-          progressed = true;
-        }
-        if (np < nq && mbar_try_wait(&sm.p_full[np & 1], (np >> 1) & 1) &&
-            mbar_try_wait(&sm.v_full[np % NV], (np / NV) & 1)) {
-          tc_fence_after();
-          const int sv = np % NV;
-          const uint64_t dv = make_sdesc(smem_u32(sm.v[sv]), kLboV, kSboV, 2u);
-          const uint32_t aP = tmem + ((np & 1) ? S_COL1 : S_COL0);
-#pragma unroll
-          for (int kk = 0; kk < KB / 16; ++kk)   // K = 16 keys per MMA: 8 TMEM columns of P, 16 rows of V
-            mma_bf16_ts(tmem + O_COL, aP + 8 * kk, dv + (16 * 128 / 16) * kk, IDESC_PV,
-                        (np > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(&sm.v_empty[sv]);
-          tc_commit(&sm.pv_done);
-          ++np;
-          progressed = true;
-        }
-        if (progressed) {
-          t_idle = 0;
-        } else {
-          if (*abort) break;
-          const uint64_t now = globaltimer_ns();
-          if (t_idle == 0) {
-            t_idle = now;
-          } else if (now - t_idle > lim) {
-            *abort = 1;
-            atomicOr(a.status, kStatusTimeout);
-            break;
-          }
-        }
+        for (int kk = 0; kk < D / 32; ++kk)
+          mma_i8_ss(dS, dq + 2 * kk, dk + 2 * kk, IDESC_QK, kk > 0 ? 1u : 0u);
+        tc_commit(&sm.s_full[n & 1]);
       }
-      tc_commit(&sm.o_full);
+      __syncwarp();
+    };
+    // PV(n): O += P(n) . V(n), A = P from TMEM (aliases S buffer n&1), K = 16 per MMA.
+    auto do_pv = [&](int n) {
+      const int sv = n % NV;
+      const uint64_t dv = dv0 + uint64_t(sv * kStrideV);
+      const uint32_t aP = tmem + ((n & 1) ? S_COL1 : S_COL0);
+      const uint32_t acc0 = n > 0 ? 1u : 0u;
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < KB / 16; ++kk)
+          mma_bf16_ts(tmem + O_COL, aP + 8 * kk, dv + (16 * 128 / 16) * kk, IDESC_PV, kk > 0 ? 1u : acc0);
+        tc_commit(&sm.v_empty[sv]);   // also tells the softmax warps that PV(n) has landed
+      }
+      __syncwarp();
+    };
+    auto wait = [&](uint64_t* bar, uint32_t par) { return __all_sync(0xffffffffu, mbar_wait(bar, par, abort, a.status, lim)); };
+    bool ok = wait(&sm.q_full, 0);
+    tc_fence_after();
+    // Blocking waits in the order events occur: QK(0), QK(1), then PV(n)
+    // (frees S buffer n&1) followed by QK(n+2). This order measured faster
+    // than an event loop polling both queues.
+    for (int n = 0; ok && n < 2 && n < N; ++n) {
+      ok = wait(&sm.k_full[n % NK], (n / NK) & 1);
+      if (ok) { tc_fence_after(); do_qk(n); }
     }
+    for (int n = 0; ok && n < N; ++n) {
+      ok = wait(&sm.p_full[n & 1], (n >> 1) & 1) && wait(&sm.v_full[n % NV], (n / NV) & 1);
+      if (!ok) break;
+      tc_fence_after();
+      do_pv(n);
+      if (n + 2 < N) {
+        ok = wait(&sm.k_full[(n + 2) % NK], ((n + 2) / NK) & 1);
+        if (ok) { tc_fence_after(); do_qk(n + 2); }
+      }
+    }
+    if (elect_one()) tc_commit(&sm.o_full);
+    __syncwarp();
   } else {
     // ------------------------------------------------------------- softmax
     const int r = tid;                                   // row within the block
@@ -316,7 +309,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     int n_cur = 0;
     // O *= alpha in TMEM once the PV product of the previous tile has landed.
     auto rescale_o = [&](float alpha) -> bool {
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done, (n_cur - 1) & 1, abort, a.status, lim))) return false;
+      // PV of the previous tile has landed once it released its V stage
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.v_empty[(n_cur - 1) % NV], ((n_cur - 1) / NV) & 1, abort,
+                                             a.status, lim)))
+        return false;
       tc_fence_after();
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
@@ -333,16 +329,16 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     for (int n = 0; n < N; ++n) {
       n_cur = n;
-      const int s = n % NV;
+      const int sk = n % NK;
       bool ok = mbar_wait(&sm.s_full[n & 1], (n >> 1) & 1, abort, a.status, lim);
-      // the tile's metadata is published with its V stage's barrier
-      ok = ok && mbar_wait(&sm.v_full[s], (n / NV) & 1, abort, a.status, lim);
+      // the tile's metadata is published with its K stage's barrier (long complete once S is in)
+      ok = ok && mbar_wait(&sm.k_full[sk], (n / NK) & 1, abort, a.status, lim);
       if (!__all_sync(0xffffffffu, ok)) {
         alive = false;
         break;
       }
       tc_fence_after();
-      const TileMeta& mt = sm.meta[s];
+      const TileMeta& mt = sm.meta[sk];
       const bool cent = mt.centroid != 0;
       const uint32_t sc = (n & 1) ? S_COL1 : S_COL0;
       uint32_t pk[32];
@@ -465,6 +461,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.p_full[n & 1]);
+      if (lane == 0) mbar_arrive(&sm.k_empty[sk]);   // done with the tile's K stage and metadata
     }
 
     // ------------------------------------------------------------ epilogue

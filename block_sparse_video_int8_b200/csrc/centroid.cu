@@ -22,7 +22,8 @@
 namespace bsva {
 namespace {
 
-// One thread per pair of columns, one "slot" of d/2 threads per key block.
+// Eight columns per thread (16-byte loads and stores), d/8 threads per key
+// block, 256/(d/8) key blocks per CTA.
 template <int D>
 __global__ void __launch_bounds__(256) centroid_kernel(const int32_t* __restrict__ k_pool,
                                                        const float* __restrict__ k_scale,
@@ -30,75 +31,83 @@ __global__ void __launch_bounds__(256) centroid_kernel(const int32_t* __restrict
                                                        int8_t* __restrict__ ck8, __nv_bfloat16* __restrict__ cv,
                                                        float* __restrict__ cfac, float* __restrict__ cbias,
                                                        int Lk, int nKB, int mode, int nCT) {
-  constexpr int TPB = D / 2;                 // threads per key block
+  constexpr int TPB = D / 8;                 // threads per key block
   constexpr int BPC = 256 / TPB;             // key blocks per CTA
   const int bh = blockIdx.y;
   const int slot = threadIdx.x / TPB;
-  const int cp = threadIdx.x % TPB;          // column pair
+  const int c8 = threadIdx.x % TPB;          // column group: columns 8*c8 .. 8*c8+7
   const int j = blockIdx.x * BPC + slot;     // key block (may be padding)
   const int nG = nCT * 32;                   // groups per head incl. padding
-  const int nblk_virtual = nG / mode;
-  if (j >= nblk_virtual) return;
+  if (j >= nG / mode) return;
   const size_t nCR = size_t(nCT) * 64;
-
   const int nj = (j < nKB) ? min(KB, Lk - j * KB) : 0;
-  // group spans (relative rows) and sizes
-  int g0[2], g1[2];
-  if (mode == 1) {
-    g0[0] = 0; g1[0] = nj; g0[1] = 0; g1[1] = 0;
-  } else {
-    g0[0] = 0; g1[0] = min(32, nj); g0[1] = min(32, nj); g1[1] = nj;
-  }
 
-  // V sums over each half of the block (fp32)
-  float sx[2] = {0.f, 0.f}, sy[2] = {0.f, 0.f};
+  // V column sums over each 32-row half of the block (fp32)
+  float sum[2][8];
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sum[h][e] = 0.f;
   if (nj > 0) {
-    const __nv_bfloat162* vp =
-        reinterpret_cast<const __nv_bfloat162*>(v + (size_t(bh) * Lk + size_t(j) * KB) * D) + cp;
-    for (int r = 0; r < nj; ++r) {
-      const float2 f = __bfloat1622float2(vp[size_t(r) * (D / 2)]);
-      const int h = (mode == 2 && r >= 32) ? 1 : 0;
-      sx[h] += f.x;
-      sy[h] += f.y;
+    const uint4* vp = reinterpret_cast<const uint4*>(v + (size_t(bh) * Lk + size_t(j) * KB) * D) + c8;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int rend = min(32 * (h + 1), nj);
+#pragma unroll 4
+      for (int r = 32 * h; r < rend; ++r) {
+        const uint4 w = __ldg(vp + size_t(r) * (D / 8));
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(b2[e]);
+          sum[h][2 * e] += f.x;
+          sum[h][2 * e + 1] += f.y;
+        }
+      }
     }
   }
   const float skj = (j < nKB) ? k_scale[size_t(bh) * nKB + j] : 0.f;
-  const int32_t* kp = (j < nKB) ? k_pool + (size_t(bh) * nKB + j) * 2 * D : nullptr;
+  const int32_t* kp = (j < nKB) ? k_pool + (size_t(bh) * nKB + j) * 2 * D + 8 * c8 : nullptr;
 
   for (int g = 0; g < mode; ++g) {
     const int G = j * mode + g;
-    const int n = g1[g] - g0[g];
-    // pool of the group
-    int32_t p0 = 0, p1 = 0;
-    if (n > 0) {
-      if (mode == 1) {
-        p0 = kp[2 * cp] + kp[D + 2 * cp];
-        p1 = kp[2 * cp + 1] + kp[D + 2 * cp + 1];
-      } else {
-        p0 = kp[g * D + 2 * cp];
-        p1 = kp[g * D + 2 * cp + 1];
-      }
+    // group rows [g0, g1) of the block: 1x64 the whole block, 2x32 its halves
+    const int g0 = (mode == 1) ? 0 : (g == 0 ? 0 : min(32, nj));
+    const int g1 = (mode == 1) ? nj : (g == 0 ? min(32, nj) : nj);
+    const int n = g1 - g0;
+    int32_t p[8];
+    float m[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      p[e] = 0;
+      if (n > 0) p[e] = (mode == 1) ? kp[e] + kp[D + e] : kp[g * D + e];
+      const float tot = (mode == 1) ? sum[0][e] + sum[1][e] : (g == 0 ? sum[0][e] : sum[1][e]);
+      m[e] = n > 0 ? tot / (float)n : 0.f;
     }
-    const size_t rhi = (size_t(bh) * nCR + 2 * size_t(G)) * D;
+    const size_t rhi = (size_t(bh) * nCR + 2 * size_t(G)) * D + 8 * c8;
     const size_t rlo = rhi + D;
-    // key rows: pool = 128*hi + lo
-    char2 hi, lo;
-    hi.x = (char)(p0 >> 7); lo.x = (char)(p0 & 127);
-    hi.y = (char)(p1 >> 7); lo.y = (char)(p1 & 127);
-    *reinterpret_cast<char2*>(ck8 + rhi + 2 * cp) = hi;
-    *reinterpret_cast<char2*>(ck8 + rlo + 2 * cp) = lo;
-    // value rows: vbar split into bf16 hi + bf16 lo
-    float mx = 0.f, my = 0.f;
-    if (n > 0) {
-      mx = sx[g] / (float)n;
-      my = sy[g] / (float)n;
+    // key rows: pool = 128*hi + lo, hi = pool >> 7 in [-64, 63], lo = pool & 127
+    uint32_t hw[2] = {0, 0}, lw[2] = {0, 0};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      hw[e >> 2] |= (uint32_t(p[e] >> 7) & 0xFF) << (8 * (e & 3));
+      lw[e >> 2] |= (uint32_t(p[e] & 127) & 0xFF) << (8 * (e & 3));
     }
-    const __nv_bfloat162 vh = __floats2bfloat162_rn(mx, my);
-    const float2 vhf = __bfloat1622float2(vh);
-    const __nv_bfloat162 vl = __floats2bfloat162_rn(mx - vhf.x, my - vhf.y);
-    *reinterpret_cast<__nv_bfloat162*>(cv + rhi + 2 * cp) = vh;
-    *reinterpret_cast<__nv_bfloat162*>(cv + rlo + 2 * cp) = vl;
-    if (cp == 0) {
+    *reinterpret_cast<uint2*>(ck8 + rhi) = make_uint2(hw[0], hw[1]);
+    *reinterpret_cast<uint2*>(ck8 + rlo) = make_uint2(lw[0], lw[1]);
+    // value rows: vbar as bf16 hi + bf16 lo
+    uint32_t vh[4], vl[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat162 h2 = __floats2bfloat162_rn(m[2 * e], m[2 * e + 1]);
+      const float2 hf = __bfloat1622float2(h2);
+      const __nv_bfloat162 l2 = __floats2bfloat162_rn(m[2 * e] - hf.x, m[2 * e + 1] - hf.y);
+      vh[e] = *reinterpret_cast<const uint32_t*>(&h2);
+      vl[e] = *reinterpret_cast<const uint32_t*>(&l2);
+    }
+    *reinterpret_cast<uint4*>(cv + rhi) = make_uint4(vh[0], vh[1], vh[2], vh[3]);
+    *reinterpret_cast<uint4*>(cv + rlo) = make_uint4(vl[0], vl[1], vl[2], vl[3]);
+    if (c8 == 0) {
       cfac[size_t(bh) * nG + G] = n > 0 ? skj / (float)n : 0.f;
       cbias[size_t(bh) * nG + G] = n > 0 ? log2f((float)n) : -INFINITY;
     }
@@ -112,7 +121,7 @@ cudaError_t launch_centroids(const bsva_shape& s, int centroid_mode, int nCT, co
                              float* cfac, float* cbias, cudaStream_t st) {
   const int nKB = (s.Lk + KB - 1) / KB;
   const int nblk_virtual = nCT * 32 / centroid_mode;
-  const int bpc = 256 / (s.d / 2);
+  const int bpc = 256 / (s.d / 8);
   dim3 grid((nblk_virtual + bpc - 1) / bpc, s.B * s.H);
   if (s.d == 128)
     centroid_kernel<128><<<grid, 256, 0, st>>>(k_pool, k_scale, v, ck8, cv, cfac, cbias, s.Lk, nKB,

@@ -20,6 +20,8 @@ constexpr uint32_t kStatusTimeout = 1u;   // workspace status bit: a wait ran ou
 // Offsets (bytes) of the regions of the caller's workspace. All 256-aligned.
 struct WsLayout {
   size_t status = 0;        // uint32 status word (+ padding to 256 B)
+  size_t scores = 0;        // fp64  [BH, nQB, nKB] routing scores (first region at a fixed offset)
+  size_t route_total = 0;   // bytes a routing call needs (status + scores)
   size_t order = 0;         // int32 [BH*nQB] work order (longest first)
   size_t ck8 = 0;           // int8  [BH, nCR, d]  centroid keys, hi/lo rows
   size_t cv = 0;            // bf16  [BH, nCR, d]  centroid values, hi/lo rows
@@ -38,6 +40,8 @@ inline WsLayout ws_layout(const bsva_shape& s, int centroid_mode) {
   const size_t BH = size_t(s.B) * s.H;
   const int nQB = (s.Lq + QB - 1) / QB, nKB = (s.Lk + KB - 1) / KB;
   size_t off = 256;
+  w.scores = off;  off = align256(off + BH * nQB * size_t(nKB) * 8);
+  w.route_total = off;
   w.order = off; off = align256(off + BH * nQB * 4);
   if (centroid_mode > 0) {
     const int groups = nKB * centroid_mode;
@@ -113,6 +117,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       return false;
     }
   }
+}
+
+// True on exactly one lane of the (converged) warp.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
 }
 
 // --------------------------------------------------------------------- TMA --
@@ -312,8 +327,8 @@ cudaError_t launch_quant_pool(const bsva_shape& s, const __nv_bfloat16* q, const
                               float* q_scale, int8_t* k8, float* k_scale, int32_t* q_pool, int32_t* k_pool,
                               cudaStream_t st);
 cudaError_t launch_route(const bsva_shape& s, double tau, const int32_t* q_pool, const int32_t* k_pool,
-                         const float* k_scale, uint8_t* kept_mask, int32_t* kept_idx, int32_t* kept_cnt,
-                         double* row_stats, cudaStream_t st);
+                         const float* k_scale, double* scores, uint8_t* kept_mask, int32_t* kept_idx,
+                         int32_t* kept_cnt, double* row_stats, cudaStream_t st);
 cudaError_t launch_centroids(const bsva_shape& s, int centroid_mode, int nCT, const int32_t* k_pool,
                              const float* k_scale, const __nv_bfloat16* v, int8_t* ck8, __nv_bfloat16* cv,
                              float* cfac, float* cbias, cudaStream_t st);

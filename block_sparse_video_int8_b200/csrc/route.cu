@@ -12,12 +12,15 @@
 // Statistics in fp64 over the routed key blocks R_i (start >= n_prefix):
 //   mu = sum s / |R|, sigma = sqrt(sum (s - mu)^2 / |R|), T = mu + tau*sigma.
 //
-// Design: one CTA of 256 threads owns TQ query-block rows of one (b, h). The
-// head's whole-block K pools stream through shared memory in tiles of 32 key
-// blocks (rows padded to d+1 words: conflict-free), each thread computes one
-// (row, key block) dot per tile, and the fp64 scores of the CTA's rows stay in
-// shared memory (TQ x nKB x 8 bytes). Then one warp per row reduces mu and
-// sigma with warp shuffles and compacts the kept list with ballots.
+// Design: two kernels.
+//  score_kernel: per head the dots are a small integer GEMM, [nQB x d] . [d x nKB]. A CTA of 256
+//   threads owns a 64 x 64 tile of (query block, key block); both pool tiles are staged in shared
+//   memory (rows padded to d+4 words: conflict-free 16-byte loads), each thread accumulates a 4 x 4
+//   block of dots (query blocks ty+16a, key blocks tx+16b) in int32 over 16 dims at a time (|q_pool|
+//   <= 16256 and |k_pool| <= 8128, so 16 products stay below 2^31) and in int64 across them, and
+//   writes the fp64 scores to the workspace, [BH, nQB, nKB].
+//  select_kernel: one warp per query-block row reduces mu and sigma with shuffles and compacts the
+//   kept list with ballots.
 #include <cmath>
 
 #include "common.cuh"
@@ -26,148 +29,169 @@ namespace bsva {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kTileJ = 32;
-constexpr int kMaxSmem = 200 * 1024;
+constexpr int kTile = 64;
 
 template <int D>
-__global__ void __launch_bounds__(kThreads) route_kernel(const int32_t* __restrict__ q_pool,
-                                                         const int32_t* __restrict__ k_pool,
-                                                         const float* __restrict__ k_scale,
-                                                         uint8_t* __restrict__ kept_mask,
-                                                         int32_t* __restrict__ kept_idx,
-                                                         int32_t* __restrict__ kept_cnt,
-                                                         double* __restrict__ row_stats, int Lk, int nQB,
-                                                         int nKB, int TQ, double tau, int tau_is_neginf,
-                                                         int n_prefix) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  double* s_score = reinterpret_cast<double*>(smem);                        // [TQ][nKB]
-  int32_t* s_q = reinterpret_cast<int32_t*>(s_score + size_t(TQ) * nKB);    // [TQ][D]
-  int32_t* s_k = s_q + TQ * D;                                              // [kTileJ][D+1]
-
-  const int bh = blockIdx.y;
-  const int i0 = blockIdx.x * TQ;
-  const int nrows = min(TQ, nQB - i0);
+__global__ void __launch_bounds__(kThreads, 2) score_kernel(const int32_t* __restrict__ q_pool,
+                                                            const int32_t* __restrict__ k_pool,
+                                                            const float* __restrict__ k_scale,
+                                                            double* __restrict__ scores, int Lk, int nQB,
+                                                            int nKB) {
+  constexpr int KS = D + 4;
+  constexpr int C4 = D / 4;
+  extern __shared__ __align__(16) int32_t sm[];
+  int32_t* sq = sm;                 // [kTile][KS] query-block pools
+  int32_t* sk = sm + kTile * KS;    // [kTile][KS] whole key-block pools (sum of the two halves)
+  const int bh = blockIdx.z, i0 = blockIdx.y * kTile, j0 = blockIdx.x * kTile;
   const int t = threadIdx.x;
 
-  for (int idx = t; idx < nrows * D; idx += kThreads)
-    s_q[idx] = q_pool[(size_t(bh) * nQB + i0) * D + idx];
-
-  // ---- scores
-  for (int j0 = 0; j0 < nKB; j0 += kTileJ) {
-    __syncthreads();
-    const int nj = min(kTileJ, nKB - j0);
-    for (int idx = t; idx < nj * D; idx += kThreads) {
-      const int jj = idx / D, c = idx % D;
-      const int32_t* p = k_pool + (size_t(bh) * nKB + j0 + jj) * 2 * D;
-      s_k[jj * (D + 1) + c] = p[c] + p[D + c];
+  for (int idx = t; idx < kTile * C4; idx += kThreads) {
+    const int r = idx / C4, c4 = idx % C4;
+    int4 a = make_int4(0, 0, 0, 0), b = make_int4(0, 0, 0, 0);
+    if (i0 + r < nQB) a = __ldg(reinterpret_cast<const int4*>(q_pool + (size_t(bh) * nQB + i0 + r) * D) + c4);
+    if (j0 + r < nKB) {
+      const int4* p = reinterpret_cast<const int4*>(k_pool + (size_t(bh) * nKB + j0 + r) * 2 * D);
+      const int4 h0 = __ldg(p + c4), h1 = __ldg(p + C4 + c4);
+      b = make_int4(h0.x + h1.x, h0.y + h1.y, h0.z + h1.z, h0.w + h1.w);
     }
-    __syncthreads();
-    for (int w = t; w < nrows * kTileJ; w += kThreads) {
-      const int r = w / kTileJ, jj = w % kTileJ;
-      if (jj >= nj) continue;
-      const int32_t* a = s_q + r * D;
-      const int32_t* b = s_k + jj * (D + 1);
-      long long acc = 0;
-#pragma unroll 16
-      for (int c = 0; c < D; ++c) acc += (long long)a[c] * b[c];
-      const int j = j0 + jj;
-      const int nj_rows = min(KB, Lk - j * KB);
-      const double prod = __dmul_rn((double)acc, (double)k_scale[size_t(bh) * nKB + j]);
-      s_score[size_t(r) * nKB + j] = __ddiv_rn(prod, (double)nj_rows);
-    }
+    *reinterpret_cast<int4*>(sq + r * KS + 4 * c4) = a;
+    *reinterpret_cast<int4*>(sk + r * KS + 4 * c4) = b;
   }
   __syncthreads();
 
-  // ---- statistics and compaction: one warp per row
-  const int warp = t >> 5, lane = t & 31;
+  const int tx = t & 15, ty = t >> 4;
+  long long acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0;
+#pragma unroll 1
+  for (int c0 = 0; c0 < D; c0 += 16) {
+    int part[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) part[a][b] = 0;
+#pragma unroll
+    for (int c = c0; c < c0 + 16; c += 4) {
+      int4 x[4], y[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) x[a] = *reinterpret_cast<const int4*>(sq + (ty + 16 * a) * KS + c);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) y[b] = *reinterpret_cast<const int4*>(sk + (tx + 16 * b) * KS + c);
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+          part[a][b] += x[a].x * y[b].x + x[a].y * y[b].y + x[a].z * y[b].z + x[a].w * y[b].w;
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] += part[a][b];
+  }
+
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const int j = j0 + tx + 16 * b;
+    if (j >= nKB) continue;
+    const double skj = (double)k_scale[size_t(bh) * nKB + j];
+    const double nj = (double)min(KB, Lk - j * KB);
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int i = i0 + ty + 16 * a;
+      if (i < nQB) scores[(size_t(bh) * nQB + i) * nKB + j] = __ddiv_rn(__dmul_rn((double)acc[a][b], skj), nj);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) select_kernel(const double* __restrict__ scores,
+                                                          uint8_t* __restrict__ kept_mask,
+                                                          int32_t* __restrict__ kept_idx,
+                                                          int32_t* __restrict__ kept_cnt,
+                                                          double* __restrict__ row_stats, int nQB, int nKB,
+                                                          double tau, int tau_is_neginf, int n_prefix) {
+  const int bh = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * (kThreads / 32) + warp;
+  if (i >= nQB) return;
   const int jr0 = (n_prefix + KB - 1) / KB;   // first routed key block
   const int nR = nKB - jr0;
-  for (int r = warp; r < nrows; r += kThreads / 32) {
-    const int i = i0 + r;
-    const double* srow = s_score + size_t(r) * nKB;
-    double sum = 0.0, mx = -INFINITY, mn = INFINITY;
-    for (int j = jr0 + lane; j < nKB; j += 32) {
-      const double v = srow[j];
-      sum += v;
-      mx = fmax(mx, v);
-      mn = fmin(mn, v);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-    }
-    const double mu = nR > 0 ? sum / nR : 0.0;
-    double ss = 0.0;
-    for (int j = jr0 + lane; j < nKB; j += 32) {
-      const double dv = srow[j] - mu;
-      ss += dv * dv;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const double sigma = nR > 0 ? sqrt(ss / nR) : 0.0;
-    const bool all_kept = tau_is_neginf || nR <= 0 || i * QB < n_prefix || mx == mn;
-    const double T = all_kept ? -INFINITY : __dadd_rn(mu, __dmul_rn(tau, sigma));
+  const size_t rowoff = (size_t(bh) * nQB + i) * nKB;
+  const double* srow = scores + rowoff;
 
-    const size_t rowoff = (size_t(bh) * nQB + i) * nKB;
-    int base = 0;
-    for (int j0 = 0; j0 < nKB; j0 += 32) {
-      const int j = j0 + lane;
-      bool keep = false;
-      if (j < nKB) keep = all_kept || j < jr0 || srow[j] >= T;
-      const unsigned bal = __ballot_sync(0xffffffffu, keep);
-      if (j < nKB) {
-        kept_mask[rowoff + j] = keep ? 1 : 0;
-        if (keep) kept_idx[rowoff + base + __popc(bal & ((1u << lane) - 1u))] = j;
-      }
-      base += __popc(bal);
+  double sum = 0.0, mx = -INFINITY, mn = INFINITY;
+  for (int j = jr0 + lane; j < nKB; j += 32) {
+    const double v = srow[j];
+    sum += v;
+    mx = fmax(mx, v);
+    mn = fmin(mn, v);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+  }
+  const double mu = nR > 0 ? sum / nR : 0.0;
+  double ss = 0.0;
+  for (int j = jr0 + lane; j < nKB; j += 32) {
+    const double dv = srow[j] - mu;
+    ss += dv * dv;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const double sigma = nR > 0 ? sqrt(ss / nR) : 0.0;
+  const bool all_kept = tau_is_neginf || nR <= 0 || i * QB < n_prefix || mx == mn;
+  const double T = all_kept ? -INFINITY : __dadd_rn(mu, __dmul_rn(tau, sigma));
+
+  int base = 0;
+  for (int j0 = 0; j0 < nKB; j0 += 32) {
+    const int j = j0 + lane;
+    bool keep = false;
+    if (j < nKB) keep = all_kept || j < jr0 || srow[j] >= T;
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (j < nKB) {
+      kept_mask[rowoff + j] = keep ? 1 : 0;
+      if (keep) kept_idx[rowoff + base + __popc(bal & ((1u << lane) - 1u))] = j;
     }
-    if (lane == 0) {
-      kept_cnt[size_t(bh) * nQB + i] = base;
-      if (row_stats) {
-        double* st = row_stats + (size_t(bh) * nQB + i) * 3;
-        st[0] = mu;
-        st[1] = sigma;
-        st[2] = T;
-      }
+    base += __popc(bal);
+  }
+  if (lane == 0) {
+    kept_cnt[size_t(bh) * nQB + i] = base;
+    if (row_stats) {
+      double* st = row_stats + (size_t(bh) * nQB + i) * 3;
+      st[0] = mu;
+      st[1] = sigma;
+      st[2] = T;
     }
   }
 }
 
 }  // namespace
 
-// Rows per CTA so that the fp64 score rows fit the shared-memory budget.
-static int route_rows_per_cta(int nKB, int d) {
-  const int fixed = kTileJ * (d + 1) * 4;
-  for (int tq = 8; tq >= 1; --tq)
-    if (size_t(tq) * nKB * 8 + size_t(tq) * d * 4 + fixed <= size_t(kMaxSmem)) return tq;
-  return 0;
-}
-
-bool route_supported(int nKB, int d) { return route_rows_per_cta(nKB, d) > 0; }
-
 cudaError_t launch_route(const bsva_shape& s, double tau, const int32_t* q_pool, const int32_t* k_pool,
-                         const float* k_scale, uint8_t* kept_mask, int32_t* kept_idx, int32_t* kept_cnt,
-                         double* row_stats, cudaStream_t st) {
+                         const float* k_scale, double* scores, uint8_t* kept_mask, int32_t* kept_idx,
+                         int32_t* kept_cnt, double* row_stats, cudaStream_t st) {
   const int nQB = (s.Lq + QB - 1) / QB, nKB = (s.Lk + KB - 1) / KB;
-  const int TQ = route_rows_per_cta(nKB, s.d);
-  if (TQ == 0) return cudaErrorInvalidValue;
-  const size_t smem = size_t(TQ) * nKB * 8 + size_t(TQ) * s.d * 4 + size_t(kTileJ) * (s.d + 1) * 4;
-  dim3 grid((nQB + TQ - 1) / TQ, s.B * s.H);
-  const int neginf = std::isinf(tau) && tau < 0;
+  const int BH = s.B * s.H;
+  const size_t smem = size_t(2) * kTile * (s.d + 4) * 4;
+  dim3 g1((nKB + kTile - 1) / kTile, (nQB + kTile - 1) / kTile, BH);
   cudaError_t e;
   if (s.d == 128) {
-    e = cudaFuncSetAttribute(route_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    e = cudaFuncSetAttribute(score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
-    route_kernel<128><<<grid, kThreads, smem, st>>>(q_pool, k_pool, k_scale, kept_mask, kept_idx, kept_cnt,
-                                                    row_stats, s.Lk, nQB, nKB, TQ, tau, neginf, s.n_prefix);
+    score_kernel<128><<<g1, kThreads, smem, st>>>(q_pool, k_pool, k_scale, scores, s.Lk, nQB, nKB);
   } else {
-    e = cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    e = cudaFuncSetAttribute(score_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
-    route_kernel<64><<<grid, kThreads, smem, st>>>(q_pool, k_pool, k_scale, kept_mask, kept_idx, kept_cnt,
-                                                   row_stats, s.Lk, nQB, nKB, TQ, tau, neginf, s.n_prefix);
+    score_kernel<64><<<g1, kThreads, smem, st>>>(q_pool, k_pool, k_scale, scores, s.Lk, nQB, nKB);
   }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int neginf = std::isinf(tau) && tau < 0;
+  dim3 g2((nQB + kThreads / 32 - 1) / (kThreads / 32), BH);
+  select_kernel<<<g2, kThreads, 0, st>>>(scores, kept_mask, kept_idx, kept_cnt, row_stats, nQB, nKB, tau, neginf,
+                                         s.n_prefix);
   return cudaGetLastError();
 }
 

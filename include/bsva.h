@@ -37,7 +37,7 @@
 extern "C" {
 #endif
 
-#define BSVA_ABI_VERSION 1
+#define BSVA_ABI_VERSION 2
 
 enum bsva_status {
   BSVA_OK = 0,
@@ -74,8 +74,14 @@ const char* bsva_last_error(void);
 /* Bytes of device workspace needed by sparse_attn_fwd (centroid_mode 1 or 2)
  * or masked_block_attn_fwd (centroid_mode 0) for shape s; 0 on a bad shape.
  * The first 256 bytes hold the device status word and must be zero before the
- * first call (bsva_check_status clears them). */
+ * first call (bsva_check_status clears them). A workspace of this size also
+ * serves sparse_attn_route: its score region comes right after the status
+ * word and no other call writes it. */
 size_t bsva_workspace_bytes(bsva_shape s, int centroid_mode);
+
+/* Bytes of device workspace sparse_attn_route needs alone (status word plus
+ * the fp64 score matrix, BH*nQB*nKB*8 bytes); 0 on a bad shape. */
+size_t bsva_route_workspace_bytes(bsva_shape s);
 
 /* Per-block symmetric INT8 quantisation and integer sum-pools, alone.
  * ("Configure Sol Sparse Attention", How it works: the proxy and the exact
@@ -109,12 +115,16 @@ int bsva_quantize_qk(bsva_shape s, const void* q, const void* k,
  *                   entries at and after kept_cnt are unspecified
  *   kept_cnt   out: int32 [B,H,nQB]
  *   row_stats  out, nullable: fp64 [B,H,nQB,3] = (mu, sigma, T); T = -inf for
- *                   rows that keep every block.                              */
+ *                   rows that keep every block.
+ *   workspace  device scratch of >= bsva_route_workspace_bytes(s) bytes,
+ *              256-aligned, owned by the caller (the scores s_ij are staged
+ *              there); BSVA_ERR_WORKSPACE if missing or too small.         */
 int sparse_attn_route(bsva_shape s, const void* q, const void* k, double tau,
                       int8_t* q8, float* q_scale, int8_t* k8, float* k_scale,
                       int32_t* q_pool, int32_t* k_pool,
                       uint8_t* kept_mask, int32_t* kept_idx, int32_t* kept_cnt,
-                      double* row_stats, bsva_stream_t stream);
+                      double* row_stats, void* workspace, size_t workspace_bytes,
+                      bsva_stream_t stream);
 
 /* Sparse attention over the routed blocks plus centroid terms
  * ("Configure Sol Sparse Attention", How it works: skipped blocks are

@@ -32,7 +32,7 @@ def test_library_builds_and_exports_every_declared_symbol():
 
 
 def test_abi_version_matches_binding():
-    assert bsva.abi_version() == bsva.ABI_VERSION == 1
+    assert bsva.abi_version() == bsva.ABI_VERSION == 2
 
 
 def test_workspace_size_arithmetic():
@@ -43,17 +43,23 @@ def test_workspace_size_arithmetic():
     assert n2 >= BH * nCT * 64 * 128 * 3 + BH * nCT * 32 * 8
     n0 = bsva.workspace_bytes(s, 0)
     assert n0 >= BH * nQB * nKB * 4
+    # routing stages its fp64 scores after the 256-byte status word; every full
+    # workspace holds that region as well
+    nr = bsva.route_workspace_bytes(s)
+    assert nr >= 256 + BH * nQB * nKB * 8
+    assert min(bsva.workspace_bytes(s, m) for m in (0, 1, 2)) >= nr
+    assert n0 >= nr + BH * nQB * nKB * 4
     with pytest.raises(bsva.BsvaError):
         bsva.workspace_bytes(bsva.Shape(1, 1, 100, 100, 96, 0), 1)   # d = 96
     with pytest.raises(bsva.BsvaError):
         bsva.workspace_bytes(s, 3)
 
 
-def _raw_route(shape, ptr=0):
+def _raw_route(shape, ptr=0, ws_bytes=1 << 30):
     lib = bsva.load()
     P = ctypes.c_void_p(ptr) if ptr else None
     return lib.sparse_attn_route(shape, P, P, ctypes.c_double(1.0), P, P, P, P, P, P, P, P, P, None,
-                                 None)
+                                 P, ws_bytes, None)
 
 
 def test_bad_arguments_return_codes_without_launching():
@@ -69,8 +75,15 @@ def test_bad_arguments_return_codes_without_launching():
     # NaN / +inf tau are rejected before any device work
     P = ctypes.c_void_p(0x1000)
     rc = lib.sparse_attn_route(good, P, P, ctypes.c_double(float("nan")), P, P, P, P, P, P, P, P, P,
-                               None, None)
+                               None, P, 1 << 30, None)
     assert rc == 1
+    # the score workspace: too small, NULL
+    assert _raw_route(good, 0x10000, ws_bytes=256) == 3
+    assert b"workspace" in lib.bsva_last_error()
+    Q = ctypes.c_void_p(0x10000)
+    rc = lib.sparse_attn_route(good, Q, Q, ctypes.c_double(1.0), Q, Q, Q, Q, Q, Q, Q, Q, Q, None,
+                               None, 1 << 30, None)
+    assert rc == 3
 
 
 def test_fwd_rejects_bad_mode_and_small_workspace():
