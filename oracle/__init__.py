@@ -17,6 +17,8 @@ What it computes, step by step, and where the source pages describe it:
                 the query block's row; dense prefix protection.
                 "Configure Sol Sparse Attention", *How it works* and *The inputs
                 that matter* (routing_threshold, prefix_policy manual).
+                Fixed-sparsity top-k selection over the same scores, prefix
+                dense ("Ref2VA VSA", *2-stage attention patch*).
 * ``attention`` softmax attention over the kept blocks exactly plus one
                 centroid term per skipped 64-token block (1x64) or two 32-token
                 centroids (2x32); and the explicit logical-block-mask entry
@@ -29,14 +31,14 @@ approximation quality of the centroid terms against dense attention
 ("parity unpinned" for that comparison only: the pages give no error figure).
 """
 from .quant import quantize_blocks, q_pools, k_half_pools, block_rows
-from .route import proxy_scores, sol_route, route_head
+from .route import proxy_scores, sol_route, route_head, topk_keep_count, topk_route
 from .attention import (centroid_groups, centroid_table, sol_attention_head,
                         masked_attention_head, physical_allowed,
                         resolve_scale)
 
 __all__ = [
     "quantize_blocks", "q_pools", "k_half_pools", "block_rows",
-    "proxy_scores", "sol_route", "route_head",
+    "proxy_scores", "sol_route", "route_head", "topk_keep_count", "topk_route",
     "centroid_groups", "centroid_table", "sol_attention_head",
     "masked_attention_head", "physical_allowed", "resolve_scale",
 ]

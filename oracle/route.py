@@ -30,6 +30,21 @@ Readings where the pages are silent or garbled:
 * Key blocks that start before n_prefix are always kept and are not in R_i.
 * Near-threshold band: a routed block with |s - T| <= 1e-6 * sigma is flagged;
   reduction order may legitimately decide it either way.
+
+Fixed-sparsity top-k routing ("Ref2VA VSA", *2-stage attention patch* and
+*Wiring it into a workflow*: top-k pruning applies only to the generated-video
+key tiles, the reference/conditioning prefix stays dense, and the recipe runs
+at sparsity 0.75). The pages' gate is a learned projection; here the same
+proxy scores as the Sol rule rank the blocks. Readings:
+
+* Each routed row keeps k = |R| - floor(sparsity * |R|) blocks (the product in
+  fp64), so "sparsity" is the skipped fraction of the routed blocks.
+* Ranking: score descending, ties to the lower key-block index.
+* Prefix query rows, an empty R, and k = |R| keep every block; key blocks
+  before n_prefix are always kept; skipped blocks keep their centroid terms
+  in the attention step exactly as under the Sol rule.
+* Row statistics: (mu, sigma) as for the Sol rule, and T = the k-th largest
+  routed score (-inf when every routed block is kept, +inf when k = 0).
 """
 import math
 
@@ -95,6 +110,50 @@ def sol_route(s, tau: float, n_prefix: int = 0):
         keep[i, ~routed] = True
         band[i, routed] = np.abs(R[i] - T) <= BAND_REL * sigma[i]
     return keep, stats, band
+
+
+def topk_keep_count(n_routed: int, sparsity: float) -> int:
+    """Routed blocks a row keeps at a fixed sparsity: |R| - floor(sparsity * |R|)."""
+    sparsity = float(sparsity)
+    if not 0.0 <= sparsity <= 1.0:
+        raise ValueError(f"sparsity must be in [0, 1], got {sparsity}")
+    return n_routed - int(math.floor(sparsity * n_routed))
+
+
+def topk_route(s, sparsity: float, n_prefix: int = 0):
+    """Fixed-sparsity top-k selection over one head's score matrix s [nQB, nKB].
+
+    Returns (keep bool [nQB, nKB], stats fp64 [nQB, 3] = (mu, sigma, T)).
+    """
+    nQB, nKB = s.shape
+    routed = (K_ROWS * np.arange(nKB)) >= n_prefix
+    ridx = np.nonzero(routed)[0]
+    nR = len(ridx)
+    k = topk_keep_count(nR, sparsity)
+    keep = np.zeros((nQB, nKB), dtype=bool)
+    stats = np.zeros((nQB, 3), dtype=np.float64)
+    R = s[:, routed]
+    if nR > 0:
+        mu = _sequential_sum(R) / nR
+        sigma = np.sqrt(_sequential_sum((R - mu[:, None]) ** 2) / nR)
+    else:
+        mu = np.zeros(nQB)
+        sigma = np.zeros(nQB)
+    for i in range(nQB):
+        if Q_ROWS * i < n_prefix or k >= nR:
+            keep[i, :] = True
+            T = -math.inf
+        else:
+            keep[i, ~routed] = True
+            if k == 0:
+                T = math.inf
+            else:
+                # primary key: score descending; secondary: key-block index ascending
+                order = ridx[np.lexsort((ridx, -s[i, ridx]))]
+                keep[i, order[:k]] = True
+                T = s[i, order[k - 1]]
+        stats[i] = (mu[i], sigma[i], T)
+    return keep, stats
 
 
 def route_head(q, k, tau: float, n_prefix: int = 0):

@@ -129,3 +129,91 @@ def test_route_independent_of_centroid_mode_and_nested_on_workload():
         keeps.append(r["keep"])
     assert (keeps[1] <= keeps[0]).all() and (keeps[2] <= keeps[1]).all()
     assert keeps[0].sum() > keeps[2].sum()
+
+
+# ------------------------------------------------------ fixed-sparsity top-k
+def test_topk_keep_count_closed_form():
+    # k = |R| - floor(sparsity * |R|): the recipe's 0.75 keeps a quarter
+    assert oracle.topk_keep_count(512, 0.75) == 128
+    assert oracle.topk_keep_count(1323, 0.75) == 331       # floor(992.25) = 992 skipped
+    assert oracle.topk_keep_count(10, 0.0) == 10
+    assert oracle.topk_keep_count(10, 1.0) == 0
+    assert oracle.topk_keep_count(0, 0.5) == 0
+    for bad in (-0.01, 1.01, float("nan")):
+        with pytest.raises(ValueError):
+            oracle.topk_keep_count(10, bad)
+
+
+def test_topk_separates_kept_from_skipped_and_breaks_ties_by_index():
+    rng = np.random.default_rng(23)
+    # coarse integer scores: many exact ties
+    s = rng.integers(-4, 5, (30, 53)).astype(np.float64)
+    for sp in (0.0, 0.3, 0.5, 0.75, 0.9, 1.0):
+        keep, stats = oracle.topk_route(s, sp)
+        k = oracle.topk_keep_count(53, sp)
+        for i in range(30):
+            kept = np.nonzero(keep[i])[0]
+            skipped = np.nonzero(~keep[i])[0]
+            assert len(kept) == k
+            if len(kept) and len(skipped):
+                lo, hi = s[i, kept].min(), s[i, skipped].max()
+                assert lo >= hi
+                # at the boundary value every kept index precedes every skipped one
+                if lo == hi:
+                    assert kept[s[i, kept] == lo].max() < skipped[s[i, skipped] == hi].min()
+                assert stats[i, 2] == lo
+            if k == 0:
+                assert stats[i, 2] == math.inf
+            if k == 53:
+                assert stats[i, 2] == -math.inf
+
+
+def test_topk_brute_force_on_tiny_rows():
+    # the kept set is the lexicographically first k-subset under (score desc, index asc)
+    import itertools
+    rng = np.random.default_rng(5)
+    for _ in range(40):
+        n = int(rng.integers(1, 8))
+        row = rng.integers(-2, 3, n).astype(np.float64)
+        for k in range(n + 1):
+            sp = (n - k) / n
+            if oracle.topk_keep_count(n, sp) != k:
+                continue
+            best = None
+            for sub in itertools.combinations(range(n), k):
+                key = (-sum(row[list(sub)]), sorted(sub))
+                if best is None or key < best[0]:
+                    best = (key, sub)
+            keep, _ = oracle.topk_route(row[None, :], sp)
+            assert sorted(np.nonzero(keep[0])[0].tolist()) == sorted(best[1])
+
+
+def test_topk_matches_sol_rule_at_the_same_count():
+    # two independent selection rules agree: with distinct scores, keeping the
+    # top m routed blocks is the Sol set whenever the Sol rule keeps m of them
+    rng = np.random.default_rng(8)
+    n = 64                                   # |R| a power of two: (n - m)/n is exact
+    for _ in range(50):
+        row = rng.standard_normal(n) * rng.uniform(0.5, 3) + rng.uniform(-2, 2)
+        for tau in (0.0, 0.5, 1.0, 1.5):
+            keep_sol, _, _ = oracle.sol_route(row[None, :], tau)
+            m = int(keep_sol.sum())
+            sp = (n - m) / n
+            assert oracle.topk_keep_count(n, sp) == m
+            keep_tk, _ = oracle.topk_route(row[None, :], sp)
+            assert (keep_tk == keep_sol).all()
+
+
+def test_topk_nested_in_sparsity_and_prefix_dense():
+    rng = np.random.default_rng(4)
+    s = rng.standard_normal((12, 40))
+    prev = None
+    for sp in (0.0, 0.25, 0.5, 0.75, 1.0):
+        keep, _ = oracle.topk_route(s, sp, n_prefix=256)     # key blocks 0-3 and query blocks 0-1 dense
+        assert keep[:, :4].all() and keep[:2].all()
+        assert (keep[2:, 4:].sum(axis=1) == oracle.topk_keep_count(36, sp)).all()
+        if prev is not None:
+            assert (keep <= prev).all()
+        prev = keep
+    keep, stats = oracle.topk_route(s, 0.5, n_prefix=64 * 40)  # nothing routed
+    assert keep.all() and (stats[:, 2] == -math.inf).all()
