@@ -43,6 +43,7 @@ import workloads  # noqa: E402
 
 METRIC = "sparse-attn ms/call + dense-equiv TFLOPS at Wan-14B-like shape; % of roofline"
 UNIT = "ms/call"
+TOPK_SPARSITY = 0.75           # the fixed-sparsity recipe's value ("Ref2VA VSA", Wiring it into a workflow)
 LAUNCHES_PER_STEP = 5          # quant_pool, score, select, centroids, attention
 
 
@@ -177,12 +178,13 @@ def route_bytes(w):
 
 # ------------------------------------------------------------ our path --
 class SolStep:
-    """Device buffers and one timed step of the Sol path for a workload and tau."""
+    """Device buffers and one timed step of the Sol path for a workload and tau
+    (or, with ``sparsity``, of the fixed-sparsity top-k routing rule)."""
 
-    def __init__(self, bsva, w, tau, Q, K, V):
-        self.bsva, self.w, self.tau = bsva, w, tau
+    def __init__(self, bsva, w, tau, Q, K, V, sparsity=None):
+        self.bsva, self.w, self.tau, self.sparsity = bsva, w, tau, sparsity
         self.Q, self.K, self.V = Q, K, V
-        self.route = bsva.sparse_attn_route(Q, K, tau, n_prefix=w.n_prefix)
+        self.route = self._route(None, None)
         self.ws = bsva.new_workspace(self.route.shape, w.centroid_mode)   # also serves routing
         self.route.scratch = None
         self.out = torch.empty_like(Q)
@@ -190,10 +192,17 @@ class SolStep:
         self.t_route = self.t_cent = self.t_attn = 0.0
         self.n = 0
 
+    def _route(self, out, ws):
+        if self.sparsity is None:
+            return self.bsva.sparse_attn_route(self.Q, self.K, self.tau, n_prefix=self.w.n_prefix, out=out,
+                                               workspace=ws)
+        return self.bsva.sparse_attn_route_topk(self.Q, self.K, self.sparsity, n_prefix=self.w.n_prefix, out=out,
+                                                workspace=ws)
+
     def step(self, timed=True):
         b, w, ev = self.bsva, self.w, self.ev
         ev[0].record()
-        b.sparse_attn_route(self.Q, self.K, self.tau, n_prefix=w.n_prefix, out=self.route, workspace=self.ws)
+        self._route(self.route, self.ws)
         ev[1].record()
         b.build_centroids(self.route, self.V, w.centroid_mode, self.ws)
         ev[2].record()
@@ -369,17 +378,21 @@ def oracle_sample(w, tau, n_route_heads, n_qblocks, seed=0):
             ref = oracle.route_head(q.float().numpy(), k.float().numpy(), tau, w.n_prefix)
             t_r += time.perf_counter() - a
             refs.append((ref, v.float().numpy()))
-        ref, v = refs[0]
-        blocks = sorted(int(x) for x in rng.choice(w.nQB, size=n_qblocks, replace=False))
-        a = time.perf_counter()
-        oracle.sol_attention_head(ref["q8"], ref["q_scale"], ref["k8"], ref["k_scale"], v, ref["keep"],
-                                  w.centroid_mode, 0.0, q_blocks=blocks)
-        t_a = time.perf_counter() - a
+        # attention units: n_qblocks query blocks spread over the routed heads
+        per_head = max(1, min(w.nQB, n_qblocks // n_route_heads))
+        t_a, n_units = 0.0, 0
+        for ref, v in refs:
+            blocks = sorted(int(x) for x in rng.choice(w.nQB, size=per_head, replace=False))
+            a = time.perf_counter()
+            oracle.sol_attention_head(ref["q8"], ref["q_scale"], ref["k8"], ref["k_scale"], v, ref["keep"],
+                                      w.centroid_mode, 0.0, q_blocks=blocks)
+            t_a += time.perf_counter() - a
+            n_units += len(blocks)
     heads = w.B * w.H
-    est_s = t_r / n_route_heads * heads + t_a / n_qblocks * heads * w.nQB
+    est_s = t_r / n_route_heads * heads + t_a / n_units * heads * w.nQB
     sample = (f"routing of {n_route_heads} head(s) (all {w.nQB} query-block rows) + attention of "
-              f"{n_qblocks} query blocks of head 0, extrapolated by unit count to {heads} heads x "
-              f"{w.nQB} query blocks; 1 thread")
+              f"{n_units} query blocks ({per_head} per routed head), extrapolated by unit count to "
+              f"{heads} heads x {w.nQB} query blocks; 1 thread")
     return est_s * 1e3, sample, time.perf_counter() - t0
 
 
@@ -466,6 +479,18 @@ def main():
                           "kept_tflops": rf["kept_tflops"], "attn_roofline_frac": rf["attn"]["frac"]})
             bsva.check_status(s2.ws)
             del s2
+        # fixed-sparsity top-k routing at the recipe's sparsity, same workload
+        s3 = SolStep(bsva, w, args.tau, Q, K, V, sparsity=TOPK_SPARSITY)
+        r3, _ = run_steps(s3, max(5, args.steps // 4), 3, dist)
+        wk = kept_work(s3.route, w)
+        rf = roofline_numbers(w, wk, r3, peaks)
+        extra["topk"] = {"sparsity": TOPK_SPARSITY, "ms_per_call": round(r3["ms"], 4),
+                         "route_ms": round(r3["route_ms"], 4), "centroid_ms": round(r3["centroid_ms"], 4),
+                         "attn_ms": round(r3["attn_ms"], 4), "measured_sparsity": round(wk["sparsity"], 4),
+                         "dense_equiv_tflops": rf["dense_equiv_tflops"], "kept_tflops": rf["kept_tflops"],
+                         "attn_roofline_frac": rf["attn"]["frac"]}
+        bsva.check_status(s3.ws)
+        del s3
         extra["lcsa_mask_entry"] = lcsa_measure(bsva, max(5, args.steps // 4), 3, dist)
     e2e = None
     if not args.quick:

@@ -9,6 +9,7 @@ Entry points (same names as the C ABI):
 
 * ``quantize_qk(q, k)``                      per-block INT8 Q/K, scales, pools
 * ``sparse_attn_route(q, k, tau, n_prefix)`` quantise + proxy score + Sol rule
+* ``sparse_attn_route_topk(q, k, sparsity, n_prefix)`` the same with fixed-sparsity top-k selection
 * ``sparse_attn_fwd(route, v, mode)``        kept blocks exact + centroids
 * ``masked_block_attn_fwd(q8, ..., mask)``   explicit logical 128x128 block mask
 """
@@ -22,7 +23,8 @@ import torch
 
 __all__ = [
     "BsvaError", "load", "lib_path", "Route", "Shape", "abi_version",
-    "workspace_bytes", "route_workspace_bytes", "quantize_qk", "sparse_attn_route", "sparse_attn_fwd",
+    "workspace_bytes", "route_workspace_bytes", "quantize_qk", "sparse_attn_route",
+    "sparse_attn_route_topk", "sparse_attn_fwd",
     "masked_block_attn_fwd", "check_status", "selftest_timeout", "new_workspace",
     "build_centroids", "sparse_attn_core",
 ]
@@ -59,6 +61,8 @@ _SIGS = {
     "bsva_workspace_bytes": (ctypes.c_size_t, [Shape, ctypes.c_int]),
     "bsva_quantize_qk": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "bsva_route_workspace_bytes": (ctypes.c_size_t, [Shape]),
+    "sparse_attn_route_topk": (ctypes.c_int, [Shape, _P, _P, ctypes.c_double, _P, _P, _P, _P, _P, _P,
+                                              _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "sparse_attn_route": (ctypes.c_int, [Shape, _P, _P, ctypes.c_double, _P, _P, _P, _P, _P, _P,
                                          _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "sparse_attn_fwd": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int,
@@ -171,6 +175,7 @@ class Route:
     kept_cnt: torch.Tensor
     row_stats: torch.Tensor | None
     scratch: torch.Tensor | None = None   # route-only workspace when the caller passes none
+    sparsity: float | None = None         # set by the fixed-sparsity top-k rule (tau is then NaN)
 
 
 def _alloc_quant(s: Shape, dev):
@@ -205,14 +210,8 @@ def route_workspace_bytes(shape: Shape) -> int:
     return n
 
 
-def sparse_attn_route(q: torch.Tensor, k: torch.Tensor, tau: float, n_prefix: int = 0,
-                      row_stats: bool = False, out: Route | None = None,
-                      workspace: torch.Tensor | None = None, stream=None) -> Route:
-    """Quantise, score and route (C ABI ``sparse_attn_route``).
-
-    ``workspace`` is a device uint8 buffer of at least ``route_workspace_bytes``
-    (a ``new_workspace`` buffer serves too); without one, a route-only buffer is
-    allocated once and kept on the returned ``Route``."""
+def _route_call(entry: str, param: float, q, k, n_prefix, row_stats, out, workspace, stream,
+                tau: float, sparsity: float | None) -> Route:
     lib = load()
     s = _shape_of(q, k, n_prefix)
     _need(q, torch.bfloat16, None, "q")
@@ -229,6 +228,7 @@ def sparse_attn_route(q: torch.Tensor, k: torch.Tensor, tau: float, n_prefix: in
                                if row_stats else None))
     else:
         out.shape, out.tau = s, tau
+    out.sparsity = sparsity
     if workspace is None:
         need = lib.bsva_route_workspace_bytes(s)   # 0 on a bad shape: the call below reports it
         if need and (out.scratch is None or out.scratch.numel() < need):
@@ -236,12 +236,34 @@ def sparse_attn_route(q: torch.Tensor, k: torch.Tensor, tau: float, n_prefix: in
         workspace = out.scratch
     if workspace is not None:
         _need(workspace, torch.uint8, None, "workspace")
-    _check(lib.sparse_attn_route(s, _ptr(q), _ptr(k), ctypes.c_double(tau), _ptr(out.q8),
-                                 _ptr(out.q_scale), _ptr(out.k8), _ptr(out.k_scale), _ptr(out.q_pool),
-                                 _ptr(out.k_pool), _ptr(out.kept_mask), _ptr(out.kept_idx),
-                                 _ptr(out.kept_cnt), _ptr(out.row_stats), _ptr(workspace),
-                                 0 if workspace is None else workspace.numel(), _stream(stream)))
+    _check(getattr(lib, entry)(s, _ptr(q), _ptr(k), ctypes.c_double(param), _ptr(out.q8),
+                               _ptr(out.q_scale), _ptr(out.k8), _ptr(out.k_scale), _ptr(out.q_pool),
+                               _ptr(out.k_pool), _ptr(out.kept_mask), _ptr(out.kept_idx),
+                               _ptr(out.kept_cnt), _ptr(out.row_stats), _ptr(workspace),
+                               0 if workspace is None else workspace.numel(), _stream(stream)))
     return out
+
+
+def sparse_attn_route(q: torch.Tensor, k: torch.Tensor, tau: float, n_prefix: int = 0,
+                      row_stats: bool = False, out: Route | None = None,
+                      workspace: torch.Tensor | None = None, stream=None) -> Route:
+    """Quantise, score and route by the Sol rule (C ABI ``sparse_attn_route``).
+
+    ``workspace`` is a device uint8 buffer of at least ``route_workspace_bytes``
+    (a ``new_workspace`` buffer serves too); without one, a route-only buffer is
+    allocated once and kept on the returned ``Route``."""
+    return _route_call("sparse_attn_route", tau, q, k, n_prefix, row_stats, out, workspace, stream,
+                       tau=tau, sparsity=None)
+
+
+def sparse_attn_route_topk(q: torch.Tensor, k: torch.Tensor, sparsity: float, n_prefix: int = 0,
+                           row_stats: bool = False, out: Route | None = None,
+                           workspace: torch.Tensor | None = None, stream=None) -> Route:
+    """Quantise, score and keep the top (1 - sparsity) of each row's routed
+    blocks (C ABI ``sparse_attn_route_topk``); workspace as for
+    ``sparse_attn_route``."""
+    return _route_call("sparse_attn_route_topk", sparsity, q, k, n_prefix, row_stats, out, workspace,
+                       stream, tau=float("nan"), sparsity=float(sparsity))
 
 
 def _out(out, shape, out_dtype, device):

@@ -228,6 +228,35 @@ int sparse_attn_route(bsva_shape s, const void* q, const void* k, double tau, in
   return ok();
 }
 
+int sparse_attn_route_topk(bsva_shape s, const void* q, const void* k, double sparsity, int8_t* q8,
+                           float* q_scale, int8_t* k8, float* k_scale, int32_t* q_pool, int32_t* k_pool,
+                           uint8_t* kept_mask, int32_t* kept_idx, int32_t* kept_cnt, double* row_stats,
+                           void* workspace, size_t workspace_bytes, bsva_stream_t stream) {
+  int rc;
+  if ((rc = check_shape(s))) return rc;
+  if (!(sparsity >= 0.0 && sparsity <= 1.0)) return fail(BSVA_ERR_INVALID_ARG, "sparsity %g is not in [0, 1]", sparsity);
+  REQUIRE_PTR(q, 16); REQUIRE_PTR(k, 16); REQUIRE_PTR(q8, 16); REQUIRE_PTR(k8, 16);
+  REQUIRE_PTR(q_scale, 4); REQUIRE_PTR(k_scale, 4); REQUIRE_PTR(q_pool, 16); REQUIRE_PTR(k_pool, 16);
+  REQUIRE_PTR(kept_mask, 1); REQUIRE_PTR(kept_idx, 4); REQUIRE_PTR(kept_cnt, 4);
+  if (row_stats && !aligned(row_stats, 8)) return fail(BSVA_ERR_INVALID_ARG, "row_stats is not 8-byte aligned");
+  const WsLayout ws = ws_layout(s, 1);
+  if ((rc = check_workspace(workspace, workspace_bytes, ws.route_total))) return rc;
+  if ((rc = check_device())) return rc;
+  // kept routed blocks per row: |R| - floor(sparsity * |R|), the product in fp64
+  const int nKB = (s.Lk + KB - 1) / KB;
+  const int nR = nKB - (s.n_prefix + KB - 1) / KB;
+  const int k_keep = nR > 0 ? nR - static_cast<int>(std::floor(sparsity * static_cast<double>(nR))) : 0;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  double* scores = reinterpret_cast<double*>(static_cast<unsigned char*>(workspace) + ws.scores);
+  cudaError_t e = launch_quant_pool(s, reinterpret_cast<const __nv_bfloat16*>(q),
+                                    reinterpret_cast<const __nv_bfloat16*>(k), q8, q_scale, k8, k_scale, q_pool,
+                                    k_pool, st);
+  if (e != cudaSuccess) return cuda_fail(e, "quant_pool launch");
+  e = launch_route_topk(s, k_keep, q_pool, k_pool, k_scale, scores, kept_mask, kept_idx, kept_cnt, row_stats, st);
+  if (e != cudaSuccess) return cuda_fail(e, "top-k route launch");
+  return ok();
+}
+
 }  // extern "C"
 
 namespace {

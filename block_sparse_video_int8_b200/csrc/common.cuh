@@ -329,6 +329,9 @@ cudaError_t launch_quant_pool(const bsva_shape& s, const __nv_bfloat16* q, const
 cudaError_t launch_route(const bsva_shape& s, double tau, const int32_t* q_pool, const int32_t* k_pool,
                          const float* k_scale, double* scores, uint8_t* kept_mask, int32_t* kept_idx,
                          int32_t* kept_cnt, double* row_stats, cudaStream_t st);
+cudaError_t launch_route_topk(const bsva_shape& s, int k_keep, const int32_t* q_pool, const int32_t* k_pool,
+                              const float* k_scale, double* scores, uint8_t* kept_mask, int32_t* kept_idx,
+                              int32_t* kept_cnt, double* row_stats, cudaStream_t st);
 cudaError_t launch_centroids(const bsva_shape& s, int centroid_mode, int nCT, const int32_t* k_pool,
                              const float* k_scale, const __nv_bfloat16* v, int8_t* ck8, __nv_bfloat16* cv,
                              float* cfac, float* cbias, cudaStream_t st);

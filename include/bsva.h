@@ -126,6 +126,32 @@ int sparse_attn_route(bsva_shape s, const void* q, const void* k, double tau,
                       double* row_stats, void* workspace, size_t workspace_bytes,
                       bsva_stream_t stream);
 
+/* Quantise + proxy score + fixed-sparsity top-k routing ("Ref2VA VSA",
+ * 2-stage attention patch: top-k pruning applies only to the generated-video
+ * key tiles and the conditioning prefix stays dense; Wiring it into a
+ * workflow: the recipe runs at sparsity 0.75). The pages rank tiles with a
+ * learned gate; this entry ranks them by the same proxy scores s_ij as
+ * sparse_attn_route, so its outputs feed sparse_attn_fwd unchanged (skipped
+ * blocks keep their centroid terms).
+ * Each row of a query block starting at or after n_prefix keeps
+ *   k = |R| - floor(sparsity * |R|)   (fp64 product)
+ * of its routed key blocks R (those starting at or after n_prefix): the k
+ * largest scores, ties to the lower key-block index. Rows before n_prefix and
+ * rows with k = |R| keep every block; key blocks before n_prefix are always
+ * kept.
+ *   sparsity   skipped fraction of the routed blocks, in [0, 1]
+ *              (BSVA_ERR_INVALID_ARG otherwise, NaN included)
+ *   row_stats  out, nullable: (mu, sigma, T) with T the k-th largest routed
+ *              score, -inf when every routed block is kept, +inf when k = 0.
+ *   Every other argument, the workspace and the outputs are as for
+ *   sparse_attn_route.                                                       */
+int sparse_attn_route_topk(bsva_shape s, const void* q, const void* k, double sparsity,
+                           int8_t* q8, float* q_scale, int8_t* k8, float* k_scale,
+                           int32_t* q_pool, int32_t* k_pool,
+                           uint8_t* kept_mask, int32_t* kept_idx, int32_t* kept_cnt,
+                           double* row_stats, void* workspace, size_t workspace_bytes,
+                           bsva_stream_t stream);
+
 /* Sparse attention over the routed blocks plus centroid terms
  * ("Configure Sol Sparse Attention", How it works: skipped blocks are
  * replaced by one 64-token centroid, or two 32-token centroids in 2x32 mode,

@@ -168,3 +168,37 @@ def masked_parity(bsva, w, mask, heads=None, q_blocks=None, softmax_scale=0.0):
                                                       allowed, softmax_scale, q_blocks=blocks)
         compare_rows(to_np(out[b, h].float()), to_np(lse[b, h]), O_ref, lse_ref, q_rows(w.Lq, blocks), rep)
     return out, lse, rep
+
+
+def topk_parity(bsva, w, sparsity, heads=None, q_blocks=None, centroid_mode=None):
+    """Top-k route + fwd on the GPU; the kept mask and T must match the oracle's
+    top-k selection over its own scores bit for bit (no tolerance band: the
+    scores are bit-exact and the ranking is a total order)."""
+    mode = centroid_mode or w.centroid_mode
+    Q, K, V = inputs(w)
+    route = bsva.sparse_attn_route_topk(Q, K, sparsity, n_prefix=w.n_prefix, row_stats=True)
+    out, lse = bsva.sparse_attn_fwd(route, V, mode, with_lse=True, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    heads = heads or [(b, h) for b in range(w.B) for h in range(w.H)]
+    rep = Report()
+    for b, h in heads:
+        q, k, v = head_np(w, b, h)
+        ref = oracle.route_head(q, k, 1.0, w.n_prefix)      # quantisation and scores
+        keep, stats = oracle.topk_route(ref["scores"], sparsity, w.n_prefix)
+        check_quant(route, ref, b, h)
+        gm = to_np(route.kept_mask[b, h]).astype(bool)
+        assert np.array_equal(gm, keep), f"top-k kept mask differs at {np.argwhere(gm != keep)[:5].tolist()}"
+        cnt = to_np(route.kept_cnt[b, h])
+        idx = to_np(route.kept_idx[b, h])
+        assert np.array_equal(cnt, keep.sum(axis=1)), "kept_cnt"
+        for i in range(keep.shape[0]):
+            assert np.array_equal(idx[i, :cnt[i]], np.nonzero(keep[i])[0]), f"kept_idx row {i}"
+        st = to_np(route.row_stats[b, h])
+        assert np.array_equal(st[:, 2], stats[:, 2]), "top-k threshold T differs"
+        scale = np.abs(stats[:, 0]) + stats[:, 1] + 1e-300
+        assert (np.abs(st[:, 0] - stats[:, 0]) <= 1e-12 * scale).all(), "mu differs"
+        blocks = list(range(w.nQB)) if q_blocks is None else [i for i in q_blocks if i < w.nQB]
+        O_ref, lse_ref = oracle.sol_attention_head(ref["q8"], ref["q_scale"], ref["k8"], ref["k_scale"], v,
+                                                   keep, mode, 0.0, q_blocks=blocks)
+        compare_rows(to_np(out[b, h].float()), to_np(lse[b, h]), O_ref, lse_ref, q_rows(w.Lq, blocks), rep)
+    return route, out, lse, rep

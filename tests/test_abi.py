@@ -86,6 +86,20 @@ def test_bad_arguments_return_codes_without_launching():
     assert rc == 3
 
 
+def test_topk_route_rejects_bad_sparsity_and_workspace():
+    lib = bsva.load()
+    good = bsva.Shape(1, 2, 256, 256, 128, 0)
+    P = ctypes.c_void_p(0x10000)
+    for sp in (-0.1, 1.5, float("nan")):
+        rc = lib.sparse_attn_route_topk(good, P, P, ctypes.c_double(sp), P, P, P, P, P, P, P, P, P, None,
+                                        P, 1 << 30, None)
+        assert rc == 1
+        assert b"sparsity" in lib.bsva_last_error()
+    rc = lib.sparse_attn_route_topk(good, P, P, ctypes.c_double(0.75), P, P, P, P, P, P, P, P, P, None,
+                                    P, 256, None)
+    assert rc == 3
+
+
 def test_fwd_rejects_bad_mode_and_small_workspace():
     lib = bsva.load()
     s = bsva.Shape(1, 2, 256, 256, 128, 0)

@@ -14,7 +14,7 @@ import torch
 import oracle
 import workloads
 from parity import (Report, assert_within, compare_rows, head_np, inputs, masked_parity, q_rows,
-                    sol_parity, to_np)
+                    sol_parity, to_np, topk_parity)
 
 pytestmark = pytest.mark.gpu
 
@@ -42,6 +42,34 @@ def test_sol_high_tau_centroid_heavy(gpu_lib):
     w = workloads.get("ragged_pe_2x32")
     route, out, lse, rep = sol_parity(gpu_lib, w, 2.5)
     assert_within(rep, "tau=2.5")
+
+
+@pytest.mark.parametrize("name,sparsity", [("ragged_pe", 0.75), ("ragged_pe_2x32", 0.5), ("ragged_d64", 0.9),
+                                           ("prefix_small", 0.75), ("cross", 0.3), ("tiny", 0.0),
+                                           ("ragged_pe", 1.0)])
+def test_topk_small_full_compare(gpu_lib, name, sparsity):
+    w = workloads.get(name)
+    route, _, _, rep = topk_parity(gpu_lib, w, sparsity)
+    assert_within(rep, f"{name} top-k sparsity={sparsity}")
+    print(f"{name} top-k sparsity={sparsity}: {rep}")
+
+
+def test_topk_ties_broken_by_index(gpu_lib):
+    # all-equal K rows: every routed score of a row ties, so the kept set is the
+    # k lowest routed indices
+    w = workloads.get("ragged_pe")
+    Q, K, _ = inputs(w)
+    K = K[:, :, :1, :].expand_as(K).contiguous()
+    r = gpu_lib.sparse_attn_route_topk(Q, K, 0.75)
+    torch.cuda.synchronize()
+    k = oracle.topk_keep_count(w.nKB, 0.75)
+    m = r.kept_mask.cpu().numpy().astype(bool)
+    # the tail block has fewer rows and so a different score; the others tie
+    q, kk, _ = head_np(w, 0, 0)
+    ref = oracle.route_head(q, to_np(K[0, 0].float()), 1.0)
+    keep, _ = oracle.topk_route(ref["scores"], 0.75)
+    assert np.array_equal(m[0, 0], keep)
+    assert (m.sum(axis=3) == k).all()
 
 
 def test_masked_small_lcsa(gpu_lib):
@@ -112,6 +140,16 @@ def test_full_lcsa(gpu_lib):
     _, _, rep = masked_parity(gpu_lib, w, workloads.block_mask(w), heads=heads,
                               q_blocks=_sample_blocks(w.nQB))
     assert_within(rep, "lcsa full")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,sparsity", [("wan14b", 0.75), ("h3", 0.75)])
+def test_full_topk(gpu_lib, name, sparsity):
+    w = workloads.get(name)
+    heads = [(0, 0), (0, w.H - 1)]
+    _, _, _, rep = topk_parity(gpu_lib, w, sparsity, heads=heads, q_blocks=_sample_blocks(w.nQB))
+    print(f"{name} top-k sparsity={sparsity}: {rep}")
+    assert_within(rep, f"{name} top-k sparsity={sparsity}")
 
 
 @pytest.mark.slow
