@@ -30,6 +30,11 @@ Readings:
   mask[b, h mod Hm, i, floor(j/2)]; exact terms only, no centroids; the
   granularity is block-level (no token-causal mask inside a block). A row with
   no allowed block gives o = 0 and lse = -inf.
+* LCSA mask from frame geometry ("FlashVSR Sparge Attention", intro: each
+  query block attends only to a small, locally causal set of key blocks; the
+  sampler builds the mask). Reading: a logical 128-token block belongs to the
+  frame of its first token, floor(128*x / frame_tokens); key block x_k is
+  allowed for query block x_q iff f_q - window <= f_k <= f_q.
 """
 import math
 
@@ -114,6 +119,20 @@ def sol_attention_head(q8, q_scale, k8, k_scale, v, keep, centroid_mode: int,
         O[r0:r1], lse[r0:r1] = _softmax_rows(np.concatenate(logits, axis=1),
                                              np.concatenate(values, axis=0))
     return O, lse
+
+
+def lcsa_mask(Lq: int, Lk: int, frame_tokens: int, window: int):
+    """Logical LCSA mask, uint8 [ceil(Lq/128), ceil(Lk/128)], built block by block."""
+    if frame_tokens <= 0 or window < 0:
+        raise ValueError("frame_tokens must be > 0 and window >= 0")
+    nq, nk = -(-Lq // 128), -(-Lk // 128)
+    m = np.zeros((nq, nk), dtype=np.uint8)
+    for xq in range(nq):
+        fq = (128 * xq) // frame_tokens
+        for xk in range(nk):
+            fk = (128 * xk) // frame_tokens
+            m[xq, xk] = 1 if fq - window <= fk <= fq else 0
+    return m
 
 
 def physical_allowed(mask_bh, nKB: int):

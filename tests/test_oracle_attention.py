@@ -142,3 +142,45 @@ def test_softmax_scale_argument():
                                      softmax_scale=0.05)
     ref = _sdpa(_dequant(r["q8"], r["q_scale"], 128), _dequant(r["k8"], r["k_scale"], 64), v, 0.05)
     assert np.abs(O - ref).max() <= 1e-12
+
+
+# ------------------------------------------------------------ LCSA geometry
+def test_lcsa_mask_density_closed_form():
+    # 8 frames of 1536 tokens (12 logical blocks each), window 2: a query block in
+    # frame f sees 12*(min(f, 2) + 1) key blocks, 144*(1 + 2 + 3*6) = 3024 of 96*96
+    m = oracle.lcsa_mask(12288, 12288, 1536, 2)
+    assert m.shape == (96, 96)
+    assert int(m.sum()) == 3024 and int(m.sum()) * 64 == 21 * 96 * 96
+    # window 0: only the block-diagonal frame squares
+    assert int(oracle.lcsa_mask(12288, 12288, 1536, 0).sum()) == 8 * 12 * 12
+
+
+def test_lcsa_mask_token_level_brute_force():
+    # a logical block takes the frame of its first token; compare with an
+    # enumeration over token positions for ragged geometries
+    rng = np.random.default_rng(3)
+    for _ in range(20):
+        Lq, Lk = int(rng.integers(1, 1500)), int(rng.integers(1, 1500))
+        F = int(rng.integers(1, 700))
+        win = int(rng.integers(0, 4))
+        m = oracle.lcsa_mask(Lq, Lk, F, win)
+        first_q = list(range(0, Lq, 128))
+        first_k = list(range(0, Lk, 128))
+        for a, tq in enumerate(first_q):
+            for b, tk in enumerate(first_k):
+                frame_q, frame_k = tq // F, tk // F
+                want = frame_k <= frame_q and frame_q - frame_k <= win
+                assert bool(m[a, b]) == want
+
+
+def test_lcsa_mask_is_causal_and_window_monotone():
+    m1 = oracle.lcsa_mask(4000, 4000, 384, 1)
+    m3 = oracle.lcsa_mask(4000, 4000, 384, 3)
+    frame = (128 * np.arange(m1.shape[0])) // 384
+    later = frame[None, :] > frame[:, None]      # key block in a later frame than the query block
+    assert (m1[later] == 0).all() and (m3[later] == 0).all()
+    assert m1[frame[None, :] == frame[:, None]].all()   # the whole own frame is visible
+    assert (m1 <= m3).all() and m3.sum() > m1.sum()
+    assert m1.diagonal().all()                  # every block sees its own frame
+    with pytest.raises(ValueError):
+        oracle.lcsa_mask(100, 100, 0, 1)
