@@ -12,6 +12,7 @@ Entry points (same names as the C ABI):
 * ``sparse_attn_route_topk(q, k, sparsity, n_prefix)`` the same with fixed-sparsity top-k selection
 * ``sparse_attn_fwd(route, v, mode)``        kept blocks exact + centroids
 * ``masked_block_attn_fwd(q8, ..., mask)``   explicit logical 128x128 block mask
+* ``build_lcsa_mask(Lq, Lk, frame_tokens, window)`` that mask from frame geometry, on the device
 """
 from __future__ import annotations
 
@@ -24,7 +25,7 @@ import torch
 __all__ = [
     "BsvaError", "load", "lib_path", "Route", "Shape", "abi_version",
     "workspace_bytes", "route_workspace_bytes", "quantize_qk", "sparse_attn_route",
-    "sparse_attn_route_topk", "sparse_attn_fwd",
+    "sparse_attn_route_topk", "build_lcsa_mask", "sparse_attn_fwd",
     "masked_block_attn_fwd", "check_status", "selftest_timeout", "new_workspace",
     "build_centroids", "sparse_attn_core",
 ]
@@ -61,6 +62,8 @@ _SIGS = {
     "bsva_workspace_bytes": (ctypes.c_size_t, [Shape, ctypes.c_int]),
     "bsva_quantize_qk": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "bsva_route_workspace_bytes": (ctypes.c_size_t, [Shape]),
+    "bsva_build_lcsa_mask": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            _P, _P]),
     "sparse_attn_route_topk": (ctypes.c_int, [Shape, _P, _P, ctypes.c_double, _P, _P, _P, _P, _P, _P,
                                               _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "sparse_attn_route": (ctypes.c_int, [Shape, _P, _P, ctypes.c_double, _P, _P, _P, _P, _P, _P,
@@ -326,6 +329,22 @@ def sparse_attn_core(route: Route, v: torch.Tensor, centroid_mode: int, workspac
                                      centroid_mode, ctypes.c_float(softmax_scale), OUT_DTYPES[out.dtype],
                                      _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
     return out
+
+
+def build_lcsa_mask(Lq: int, Lk: int, frame_tokens: int, window_frames: int, batch: int = 1,
+                    out: torch.Tensor | None = None, device=None, stream=None) -> torch.Tensor:
+    """The LCSA logical mask from frame geometry, built on the device (C ABI
+    ``bsva_build_lcsa_mask``): uint8 [batch, 1, ceil(Lq/128), ceil(Lk/128)]."""
+    lib = load()
+    shape = (max(batch, 0), 1, -(-Lq // 128) if Lq > 0 else 0, -(-Lk // 128) if Lk > 0 else 0)
+    if out is None:
+        m = torch.empty(shape, dtype=torch.uint8, device=device or "cuda")
+    else:
+        _need(out, torch.uint8, shape, "out")
+        m = out
+    _check(lib.bsva_build_lcsa_mask(Lq, Lk, frame_tokens, window_frames, batch,
+                                    _ptr(m) if m.numel() else None, _stream(stream)))
+    return m
 
 
 def masked_block_attn_fwd(q8, q_scale, k8, k_scale, v, block_mask, softmax_scale: float = 0.0,

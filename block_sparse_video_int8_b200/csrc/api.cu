@@ -257,6 +257,20 @@ int sparse_attn_route_topk(bsva_shape s, const void* q, const void* k, double sp
   return ok();
 }
 
+int bsva_build_lcsa_mask(int Lq, int Lk, int frame_tokens, int window_frames, int batch, uint8_t* mask,
+                         bsva_stream_t stream) {
+  if (Lq < 1 || Lk < 1 || batch < 1) return fail(BSVA_ERR_INVALID_ARG, "Lq, Lk and batch must be >= 1");
+  if (frame_tokens < 1) return fail(BSVA_ERR_INVALID_ARG, "frame_tokens = %d must be >= 1", frame_tokens);
+  if (window_frames < 0) return fail(BSVA_ERR_INVALID_ARG, "window_frames = %d must be >= 0", window_frames);
+  REQUIRE_PTR(mask, 1);
+  int rc;
+  if ((rc = check_device())) return rc;
+  cudaError_t e = launch_lcsa_mask(Lq, Lk, frame_tokens, window_frames, batch, mask,
+                                   reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lcsa mask launch");
+  return ok();
+}
+
 }  // extern "C"
 
 namespace {

@@ -335,6 +335,8 @@ cudaError_t launch_route_topk(const bsva_shape& s, int k_keep, const int32_t* q_
 cudaError_t launch_centroids(const bsva_shape& s, int centroid_mode, int nCT, const int32_t* k_pool,
                              const float* k_scale, const __nv_bfloat16* v, int8_t* ck8, __nv_bfloat16* cv,
                              float* cfac, float* cbias, cudaStream_t st);
+cudaError_t launch_lcsa_mask(int Lq, int Lk, int frame_tokens, int window, int batch, uint8_t* mask,
+                             cudaStream_t st);
 cudaError_t launch_mask_expand(const bsva_shape& s, const uint8_t* block_mask, int mask_heads, int32_t* kept_idx,
                                int32_t* kept_cnt, cudaStream_t st);
 cudaError_t launch_attention(const AttnArgs& a, const AttnMaps& maps, cudaStream_t st);

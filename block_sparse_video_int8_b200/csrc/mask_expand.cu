@@ -8,6 +8,14 @@
 //
 // One warp per (b, h, query block) row; ballots compact the allowed indices
 // in ascending order.
+//
+// lcsa_mask_kernel builds the logical mask itself from frame geometry
+// ("FlashVSR Sparge Attention", intro: each query block attends only to a
+// small, locally causal set of key blocks): a 128-token block belongs to the
+// frame of its first token, floor(128 x / frame_tokens), and key block x_k is
+// allowed for query block x_q iff f_q - window <= f_k <= f_q.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace bsva {
@@ -35,7 +43,26 @@ __global__ void __launch_bounds__(256) mask_expand_kernel(const uint8_t* __restr
   if (lane == 0) kcnt[row] = base;
 }
 
+__global__ void __launch_bounds__(256) lcsa_mask_kernel(uint8_t* __restrict__ mask, int nQB, int nLK, int frame_tokens,
+                                                        int window, size_t total) {
+  for (size_t idx = size_t(blockIdx.x) * blockDim.x + threadIdx.x; idx < total; idx += size_t(gridDim.x) * blockDim.x) {
+    const int xk = int(idx % nLK);
+    const int xq = int((idx / nLK) % nQB);
+    const long long fq = (128LL * xq) / frame_tokens, fk = (128LL * xk) / frame_tokens;
+    mask[idx] = (fk <= fq && fq - fk <= window) ? 1 : 0;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_lcsa_mask(int Lq, int Lk, int frame_tokens, int window, int batch, uint8_t* mask,
+                             cudaStream_t st) {
+  const int nQB = (Lq + QB - 1) / QB, nLK = (Lk + 127) / 128;
+  const size_t total = size_t(batch) * nQB * nLK;
+  const unsigned grid = unsigned(std::min<size_t>((total + 255) / 256, 148 * 16));
+  lcsa_mask_kernel<<<grid, 256, 0, st>>>(mask, nQB, nLK, frame_tokens, window, total);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_mask_expand(const bsva_shape& s, const uint8_t* block_mask, int mask_heads, int32_t* kept_idx,
                                int32_t* kept_cnt, cudaStream_t st) {

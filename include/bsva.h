@@ -197,6 +197,20 @@ int bsva_sparse_attn_core(bsva_shape s, const int8_t* q8, const float* q_scale,
                           float* lse, void* workspace, size_t workspace_bytes,
                           bsva_stream_t stream);
 
+/* The LCSA logical block mask built on the device from frame geometry
+ * ("FlashVSR Sparge Attention", intro: local causal sparse attention, each
+ * query block attends only to a small, locally causal set of key blocks; the
+ * sampler builds that mask). A logical 128-token block belongs to the frame
+ * of its first token, f(x) = floor(128 x / frame_tokens); key block x_k is
+ * allowed for query block x_q iff f(x_q) - window_frames <= f(x_k) <= f(x_q).
+ *   mask   out: uint8 [batch, 1, ceil(Lq/128), ceil(Lk/128)] (every batch
+ *          entry the same), ready for masked_block_attn_fwd with
+ *          mask_heads = 1.
+ *   BSVA_ERR_INVALID_ARG for Lq, Lk, batch or frame_tokens < 1,
+ *   window_frames < 0 or a NULL mask; asynchronous on stream otherwise.     */
+int bsva_build_lcsa_mask(int Lq, int Lk, int frame_tokens, int window_frames,
+                         int batch, uint8_t* mask, bsva_stream_t stream);
+
 /* Attention over an explicit logical block mask, exact terms only
  * ("FlashVSR Sparge Attention", How it works: routing on logical
  * 128-query x 128-key blocks, converted to the kernel's physical geometry

@@ -100,6 +100,14 @@ def test_topk_route_rejects_bad_sparsity_and_workspace():
     assert rc == 3
 
 
+def test_lcsa_builder_rejects_bad_geometry():
+    lib = bsva.load()
+    P = ctypes.c_void_p(0x10000)
+    for args in ((0, 100, 64, 1, 1), (100, 100, 0, 1, 1), (100, 100, 64, -1, 1), (100, 100, 64, 1, 0)):
+        assert lib.bsva_build_lcsa_mask(*args, P, None) == 1
+    assert lib.bsva_build_lcsa_mask(100, 100, 64, 1, 1, None, None) == 1
+
+
 def test_fwd_rejects_bad_mode_and_small_workspace():
     lib = bsva.load()
     s = bsva.Shape(1, 2, 256, 256, 128, 0)

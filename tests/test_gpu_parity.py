@@ -78,6 +78,27 @@ def test_masked_small_lcsa(gpu_lib):
     assert_within(rep, "lcsa_small")
 
 
+@pytest.mark.parametrize("Lq,Lk,F,win,batch", [(12288, 12288, 1536, 2, 1), (1000, 1304, 300, 1, 2),
+                                               (4000, 700, 128, 0, 1), (129, 5000, 1, 3, 3)])
+def test_lcsa_device_mask_matches_oracle(gpu_lib, Lq, Lk, F, win, batch):
+    m = gpu_lib.build_lcsa_mask(Lq, Lk, F, win, batch=batch)
+    torch.cuda.synchronize()
+    ref = oracle.lcsa_mask(Lq, Lk, F, win)
+    got = m.cpu().numpy()
+    assert got.shape == (batch, 1) + ref.shape
+    for b in range(batch):
+        assert np.array_equal(got[b, 0], ref)
+
+
+def test_masked_small_lcsa_device_mask(gpu_lib):
+    # the mask path end to end with the device-built mask
+    w = workloads.get("lcsa_small")
+    m = gpu_lib.build_lcsa_mask(w.Lq, w.Lk, w.frame_tokens, w.lcsa_window, batch=w.B).cpu()
+    assert np.array_equal(m[0, 0].numpy(), oracle.lcsa_mask(w.Lq, w.Lk, w.frame_tokens, w.lcsa_window))
+    _, _, rep = masked_parity(gpu_lib, w, m)
+    assert_within(rep, "lcsa_small device mask")
+
+
 def test_masked_per_head_random_mask_with_empty_rows(gpu_lib):
     w = workloads.get("cross")
     rng = np.random.default_rng(5)
