@@ -501,7 +501,7 @@ def main():
         e2e = e2e_measure(bsva, w, args.tau, Qp, Kp, Vp, max(3, args.steps // 10), 2, dist)
     cpu = None
     if rank == 0 and world == 1 and not args.quick:
-        v_ms, sample, secs = oracle_sample(w, args.tau, 4, 384)
+        v_ms, sample, secs = oracle_sample(w, args.tau, 8, 768)
         cpu = {"value": round(v_ms, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": sample + f" ({secs:.1f} s of CPU work)"}
 
