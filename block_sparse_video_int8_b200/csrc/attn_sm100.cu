@@ -13,11 +13,13 @@
 //              2^8, and runs the epilogue O / l.
 //   warp 4     TMA producer: Q tile once, then K (int8) tiles with their
 //              per-tile metadata into a 4-stage ring (freed by the softmax
-//              warps once they are done with the tile) one tile ahead of V
-//              (bf16) tiles in a 3-stage ring (freed when PV is done): first
-//              the kept blocks, then the centroid tiles.
+//              warps once they are done with the tile), first the kept
+//              blocks, then the centroid tiles.
 //   warp 5     TMEM owner (alloc/dealloc) and MMA issuer (the warp runs the
-//              schedule, one elected lane issues):
+//              schedule, one elected lane issues); it also loads the V
+//              (bf16) tiles into a 3-stage ring, two tiles ahead of PV, as
+//              soon as a stage's last PV has landed, so that K and V loads
+//              (about 1.5 us each here) never wait for one another:
 //              S = Q8 . K8^T with tcgen05.mma kind::i8 (M=128, N=64, int32
 //              accumulate) and O += P . V with kind::f16 (A = P from TMEM,
 //              B = V from shared memory, fp32 accumulate). S is double
@@ -36,6 +38,7 @@ namespace {
 
 constexpr int NK = 4;           // K tile + metadata stages (freed once the softmax is done with the tile)
 constexpr int NV = 3;           // V tile stages (freed once PV is done)
+constexpr int NR = 8;           // V row slots passed from the producer to the V loads
 constexpr int kThreads = 192;
 constexpr float kRescaleLog2 = 8.0f;   // lazy O rescale threshold (factor 256)
 constexpr uint32_t kTmemCols = 256;
@@ -57,6 +60,7 @@ struct __align__(1024) Smem {
   int8_t k[NK][KB * D];
   __nv_bfloat16 v[NV][KB * D];
   TileMeta meta[NK];
+  int vrow[NR];         // first V row of tile t at [t % NR], written before K(t)'s barrier is armed
   uint64_t q_full;
   uint64_t k_full[NK];
   uint64_t k_empty[NK];
@@ -145,8 +149,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
-    // One warp, two cursors: the K tile (and metadata) of step n+1 is issued
-    // before the V tile of step n, so K runs a tile ahead. Kept indices and
+    // K tiles (and metadata) as soon as their stage is free. Kept indices and
     // their scales are fetched 32 tiles at a time, one per lane; centroid
     // metadata is fetched a tile ahead, one group per lane. Lane 0 issues TMA.
     const float sqs = a.q_scale[row_item] * a.scale_log2e;
@@ -163,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     int chunk_j = 0;          // kept index of tile (32*c + lane) of the current chunk
     float chunk_f = 0.f;
-    int j_cur = 0, j_next = 0;   // key block of the V step's tile and of the K step's tile
+    int j_next = 0;              // key block of the K step's tile
     float cf_next = 0.f, cb_next = 0.f;   // centroid metadata of the next centroid tile
     bool ok = true;
 
@@ -206,6 +209,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (lane == 0) mt.centroid = 1;
         if (t + 1 < N) cent_meta(tc + 1, cf_next, cb_next);   // prefetch the next centroid tile
       }
+      if (lane == 0) sm.vrow[t % NR] = row;
       __syncwarp();   // the metadata is published by lane 0's arrive on the stage's barrier
       if (lane == 0) {
         mbar_arrive_expect_tx(&sm.k_full[sk], KB * D);
@@ -213,26 +217,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       return true;
     };
-    auto v_step = [&](int t) -> bool {
-      const int sv = t % NV;
-      if (t >= NV && !__all_sync(0xffffffffu, mbar_wait(&sm.v_empty[sv], ((t / NV) - 1) & 1, abort, a.status, lim)))
-        return false;
-      const int row = t < n_exact ? j_cur * KB : (t - n_exact) * KB;
-      if (lane == 0) {
-        const CUtensorMap* mv = t < n_exact ? &maps.v : &maps.cv;
-        mbar_arrive_expect_tx(&sm.v_full[sv], KB * D * 2);
-        tma_load_3d(sm.v[sv], mv, 0, row, bh, &sm.v_full[sv]);
-        if (D == 128) tma_load_3d(sm.v[sv] + KB * 64, mv, 64, row, bh, &sm.v_full[sv]);
-      }
-      return true;
-    };
-
-    ok = k_step(0);
-    for (int n = 0; ok && n < N; ++n) {
-      j_cur = j_next;
-      if (n + 1 < N) ok = k_step(n + 1);
-      if (ok) ok = v_step(n);
-    }
+    for (int t = 0; ok && t < N; ++t) ok = k_step(t);
   } else if (warp == 5) {
     // ---------------------------------------------------------- MMA issuer
     // K-major INT8 tiles: rows of D bytes, 8-row groups of 8*D bytes.
@@ -278,6 +263,21 @@ __global__ void __launch_bounds__(kThreads, 2)
       __syncwarp();
     };
     auto wait = [&](uint64_t* bar, uint32_t par) { return __all_sync(0xffffffffu, mbar_wait(bar, par, abort, a.status, lim)); };
+    // V(t) into stage t % NV once PV(t - NV) has landed; its row was published
+    // with K(t)'s barrier, which this warp has already waited on.
+    auto v_load = [&](int t) -> bool {
+      const int sv = t % NV;
+      if (t >= NV && !wait(&sm.v_empty[sv], ((t / NV) - 1) & 1)) return false;
+      if (lane == 0) {
+        const int row = sm.vrow[t % NR];
+        const CUtensorMap* mv = t < n_exact ? &maps.v : &maps.cv;
+        mbar_arrive_expect_tx(&sm.v_full[sv], KB * D * 2);
+        tma_load_3d(sm.v[sv], mv, 0, row, bh, &sm.v_full[sv]);
+        if (D == 128) tma_load_3d(sm.v[sv] + KB * 64, mv, 64, row, bh, &sm.v_full[sv]);
+      }
+      __syncwarp();
+      return true;
+    };
     bool ok = wait(&sm.q_full, 0);
     tc_fence_after();
     // Blocking waits in the order events occur: QK(0), QK(1), then PV(n)
@@ -286,6 +286,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int n = 0; ok && n < 2 && n < N; ++n) {
       ok = wait(&sm.k_full[n % NK], (n / NK) & 1);
       if (ok) { tc_fence_after(); do_qk(n); }
+      if (ok) ok = v_load(n);
     }
     for (int n = 0; ok && n < N; ++n) {
       ok = wait(&sm.p_full[n & 1], (n >> 1) & 1) && wait(&sm.v_full[n % NV], (n / NV) & 1);
@@ -294,7 +295,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       do_pv(n);
       if (n + 2 < N) {
         ok = wait(&sm.k_full[(n + 2) % NK], ((n + 2) / NK) & 1);
-        if (ok) { tc_fence_after(); do_qk(n + 2); }
+        // no second fence: the one after the p_full wait above already orders this
+        // QK's S writes after the softmax warps' loads of that buffer, and the K
+        // tile arrives by TMA under its own barrier
+        if (ok) do_qk(n + 2);
+        if (ok) ok = v_load(n + 2);   // needs PV(n - 1), issued one step ago
       }
     }
     if (elect_one()) tc_commit(&sm.o_full);
