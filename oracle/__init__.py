@@ -30,14 +30,14 @@ torch, exact-arithmetic statistics). The one quantity left unpinned is the
 approximation quality of the centroid terms against dense attention
 ("parity unpinned" for that comparison only: the pages give no error figure).
 """
-from .quant import quantize_blocks, q_pools, k_half_pools, block_rows
+from .quant import quantize_blocks, dequantize_blocks, q_pools, k_half_pools, block_rows
 from .route import proxy_scores, sol_route, route_head, topk_keep_count, topk_route
 from .attention import (centroid_groups, centroid_table, sol_attention_head,
                         masked_attention_head, physical_allowed, lcsa_mask,
                         resolve_scale)
 
 __all__ = [
-    "quantize_blocks", "q_pools", "k_half_pools", "block_rows",
+    "quantize_blocks", "dequantize_blocks", "q_pools", "k_half_pools", "block_rows",
     "proxy_scores", "sol_route", "route_head", "topk_keep_count", "topk_route",
     "centroid_groups", "centroid_table", "sol_attention_head", "lcsa_mask",
     "masked_attention_head", "physical_allowed", "resolve_scale",

@@ -18,6 +18,10 @@ state neither the block size nor the rounding; the readings used here are:
   block, and per 64-row K block one per 32-row half. The halves of a tail K
   block with n valid rows are rows [0, min(32, n)) and [32, n); an empty half
   sums to zero.
+* INT8 V ("FlashVSR Kitchen Sparse Attention", intro: the streaming cache
+  keeps K/V as INT8 and the sparse kernel consumes it without rebuilding bf16
+  tensors): V uses the K quantiser, 64-row blocks, and its dequantised value
+  is x8 * s (fp64 here), the tensor the attention then weights.
 """
 import numpy as np
 
@@ -72,4 +76,13 @@ def k_half_pools(k8):
         mid = min(t1, t0 + 32)
         out[j, 0] = k8[t0:mid].astype(np.int64).sum(axis=0)
         out[j, 1] = k8[mid:t1].astype(np.int64).sum(axis=0)
+    return out
+
+
+def dequantize_blocks(x8, scale, rows: int):
+    """fp64 values x8 * s of a per-block INT8 tensor [L, d] with scales [nBlocks]."""
+    x8 = np.asarray(x8)
+    out = np.empty(x8.shape, dtype=np.float64)
+    for b, (t0, t1) in enumerate(block_rows(x8.shape[0], rows)):
+        out[t0:t1] = x8[t0:t1].astype(np.float64) * float(scale[b])
     return out

@@ -125,3 +125,22 @@ def test_tail_half_can_be_empty():
     assert PK.shape[0] == 21
     assert (PK[20, 1] == 0).all()
     assert (PK[20, 0] == k8[1280:1304].astype(np.int64).sum(0)).all()
+
+
+def test_dequantised_v_within_half_a_step_and_exact_on_grid():
+    # INT8 V reuses the K quantiser; its dequantised value x8*s is within half a
+    # quantisation step of the input (plus the fp32 rounding of x/s), and exact
+    # for inputs that already sit on the grid
+    rng = np.random.default_rng(12)
+    v = (rng.standard_normal((1000, 64)) * rng.uniform(0.1, 3, (1000, 1))).astype(np.float32)
+    v8, sv = oracle.quantize_blocks(v, oracle.quant.K_ROWS)
+    deq = oracle.dequantize_blocks(v8, sv, oracle.quant.K_ROWS)
+    for b, (t0, t1) in enumerate(oracle.block_rows(1000, 64)):
+        err = np.abs(deq[t0:t1] - v[t0:t1].astype(np.float64))
+        assert (err <= sv[b] * (0.5 + 2.0 ** -17) + 1e-30).all()
+    # values n*s with |n| <= 127 come back exactly (n = 127 sets amax)
+    s = np.float32(0.03125)
+    n = rng.integers(-127, 128, (64, 32)).astype(np.float32)
+    n[0, 0] = 127
+    x8, sx = oracle.quantize_blocks(n * s, 64)
+    assert np.array_equal(oracle.dequantize_blocks(x8, sx, 64), (n * s).astype(np.float64))
