@@ -331,7 +331,7 @@ def e2e_measure(bsva, w, tau, Qh, Kh, Vh, steps, warmup, dist):
     return {"value": round(ms, 4), "unit": UNIT, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
 
 
-def lcsa_measure(bsva, steps, warmup, dist):
+def lcsa_measure(bsva, steps, warmup, dist, int8_v=False):
     w = workloads.get("lcsa")
     Q, K, V = [x.cuda() for x in workloads.batch_qkv(w)]
     mask = bsva.build_lcsa_mask(w.Lq, w.Lk, w.frame_tokens, w.lcsa_window, batch=w.B)
@@ -339,12 +339,19 @@ def lcsa_measure(bsva, steps, warmup, dist):
     ws = bsva.new_workspace(bsva.Shape(w.B, w.H, w.Lq, w.Lk, w.d, 0), 0)
     out = torch.empty_like(Q)
 
+    vq = bsva.quantize_v(V) if int8_v else None
+
     def one():
         # the whole mask path: LCSA mask from frame geometry, quantise, mask attention
         bsva.build_lcsa_mask(w.Lq, w.Lk, w.frame_tokens, w.lcsa_window, batch=w.B, out=mask)
         bsva.quantize_qk(Q, K, out=qk)
-        bsva.masked_block_attn_fwd(qk["q8"], qk["q_scale"], qk["k8"], qk["k_scale"], V, mask, workspace=ws,
-                                   out=out)
+        if int8_v:
+            bsva.quantize_v(V, out=vq)
+            bsva.masked_block_attn_fwd_v8(qk["q8"], qk["q_scale"], qk["k8"], qk["k_scale"], vq["v8"],
+                                          vq["v_scale"], mask, workspace=ws, out=out)
+        else:
+            bsva.masked_block_attn_fwd(qk["q8"], qk["q_scale"], qk["k8"], qk["k_scale"], V, mask, workspace=ws,
+                                       out=out)
 
     for _ in range(warmup):
         one()
@@ -359,7 +366,8 @@ def lcsa_measure(bsva, steps, warmup, dist):
     allowed = int(mask.sum().item()) * 128 * 128 * w.H * w.B       # logical pairs (all blocks full here)
     bsva.check_status(ws)
     return {"workload": "lcsa: B=1 H=12 d=128 L=12288 (8 frames x 32x48), window [f-2, f]; "
-                        "device mask build + quantise + mask attention",
+                        "device mask build + quantise" + (" Q, K and V (INT8 V)" if int8_v else "")
+                        + " + mask attention",
             "ms_per_call": round(ms, 4), "kept_frac": round(int(mask.sum().item()) / mask.numel(), 6),
             "kept_tflops": round(4.0 * w.d * allowed / (ms * 1e-3) / 1e12, 2),
             "dense_equiv_tflops": round(w.dense_flops() / (ms * 1e-3) / 1e12, 2)}
@@ -495,6 +503,7 @@ def main():
         bsva.check_status(s3.ws)
         del s3
         extra["lcsa_mask_entry"] = lcsa_measure(bsva, max(5, args.steps // 4), 3, dist)
+        extra["lcsa_mask_entry_int8_v"] = lcsa_measure(bsva, max(5, args.steps // 4), 3, dist, int8_v=True)
     e2e = None
     if not args.quick:
         Qp, Kp, Vp = Qh.pin_memory(), Kh.pin_memory(), Vh.pin_memory()

@@ -13,6 +13,7 @@ Entry points (same names as the C ABI):
 * ``sparse_attn_fwd(route, v, mode)``        kept blocks exact + centroids
 * ``masked_block_attn_fwd(q8, ..., mask)``   explicit logical 128x128 block mask
 * ``build_lcsa_mask(Lq, Lk, frame_tokens, window)`` that mask from frame geometry, on the device
+* ``quantize_v(v)``, ``masked_block_attn_fwd_v8(...)`` the mask entry on an INT8 V
 """
 from __future__ import annotations
 
@@ -25,7 +26,7 @@ import torch
 __all__ = [
     "BsvaError", "load", "lib_path", "Route", "Shape", "abi_version",
     "workspace_bytes", "route_workspace_bytes", "quantize_qk", "sparse_attn_route",
-    "sparse_attn_route_topk", "build_lcsa_mask", "sparse_attn_fwd",
+    "sparse_attn_route_topk", "build_lcsa_mask", "quantize_v", "masked_block_attn_fwd_v8", "sparse_attn_fwd",
     "masked_block_attn_fwd", "check_status", "selftest_timeout", "new_workspace",
     "build_centroids", "sparse_attn_core",
 ]
@@ -79,6 +80,10 @@ _SIGS = {
     "masked_block_attn_fwd_noalloc": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, _P, ctypes.c_int,
                                                      ctypes.c_float, ctypes.c_int, _P, _P, _P]),
     "bsva_check_status": (ctypes.c_int, [_P, _P]),
+    "bsva_quantize_v": (ctypes.c_int, [Shape, _P, _P, _P, _P]),
+    "masked_block_attn_fwd_v8": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int,
+                                                ctypes.c_float, ctypes.c_int, _P, _P, _P, ctypes.c_size_t,
+                                                _P]),
     "bsva_selftest_timeout": (ctypes.c_int, [_P, ctypes.c_size_t, ctypes.c_longlong, _P]),
 }
 
@@ -347,32 +352,64 @@ def build_lcsa_mask(Lq: int, Lk: int, frame_tokens: int, window_frames: int, bat
     return m
 
 
-def masked_block_attn_fwd(q8, q_scale, k8, k_scale, v, block_mask, softmax_scale: float = 0.0,
-                          with_lse: bool = False, workspace=None, out=None, lse=None,
-                          out_dtype=torch.bfloat16, stream=None):
-    """Attention over an explicit logical 128x128 block mask (C ABI ``masked_block_attn_fwd``)."""
+def _masked_call(entry, q8, q_scale, k8, k_scale, v_args, v_like, block_mask, softmax_scale, with_lse,
+                 workspace, out, lse, out_dtype, stream):
     lib = load()
     B, H, Lq, d = q8.shape
     Lk = k8.shape[2]
     s = Shape(B, H, Lq, Lk, d, 0)
     _need(q8, torch.int8, None, "q8")
     _need(k8, torch.int8, (B, H, Lk, d), "k8")
-    _need(v, torch.bfloat16, (B, H, Lk, d), "v")
     _need(block_mask, torch.uint8, None, "block_mask")
     if block_mask.dim() != 4 or block_mask.shape[0] != B or block_mask.shape[2:] != (-(-Lq // 128), -(-Lk // 128)):
         raise ValueError(f"block_mask shape {tuple(block_mask.shape)} is not [B, Hm, nQB, nLK]")
     mask_heads = block_mask.shape[1]
     if workspace is None:
-        workspace = new_workspace(s, 0, v.device)
-    out = _out(out, (B, H, Lq, d), out_dtype, v.device)
+        workspace = new_workspace(s, 0, v_like.device)
+    out = _out(out, (B, H, Lq, d), out_dtype, v_like.device)
     if with_lse and lse is None:
-        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=v.device)
-    _check(lib.masked_block_attn_fwd(s, _ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(k_scale), _ptr(v),
-                                     _ptr(block_mask), mask_heads, ctypes.c_float(softmax_scale),
-                                     OUT_DTYPES[out.dtype], _ptr(out), _ptr(lse), _ptr(workspace),
-                                     workspace.numel(),
-                                     _stream(stream)))
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=v_like.device)
+    _check(getattr(lib, entry)(s, _ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(k_scale), *[_ptr(t) for t in v_args],
+                               _ptr(block_mask), mask_heads, ctypes.c_float(softmax_scale),
+                               OUT_DTYPES[out.dtype], _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+                               _stream(stream)))
     return (out, lse) if with_lse else out
+
+
+def masked_block_attn_fwd(q8, q_scale, k8, k_scale, v, block_mask, softmax_scale: float = 0.0,
+                          with_lse: bool = False, workspace=None, out=None, lse=None,
+                          out_dtype=torch.bfloat16, stream=None):
+    """Attention over an explicit logical 128x128 block mask (C ABI ``masked_block_attn_fwd``)."""
+    B, H, _, d = q8.shape
+    _need(v, torch.bfloat16, (B, H, k8.shape[2], d), "v")
+    return _masked_call("masked_block_attn_fwd", q8, q_scale, k8, k_scale, (v,), v, block_mask, softmax_scale,
+                        with_lse, workspace, out, lse, out_dtype, stream)
+
+
+def quantize_v(v: torch.Tensor, out: dict | None = None, stream=None) -> dict:
+    """Per-64-row-block INT8 V and its scales (C ABI ``bsva_quantize_v``)."""
+    lib = load()
+    _need(v, torch.bfloat16, None, "v")
+    if v.dim() != 4:
+        raise ValueError("v must be [B, H, Lk, d]")
+    B, H, Lk, d = v.shape
+    s = Shape(B, H, Lk, Lk, d, 0)
+    o = out or dict(v8=torch.empty(v.shape, dtype=torch.int8, device=v.device),
+                    v_scale=torch.empty((B, H, -(-Lk // 64)), dtype=torch.float32, device=v.device))
+    _check(lib.bsva_quantize_v(s, _ptr(v), _ptr(o["v8"]), _ptr(o["v_scale"]), _stream(stream)))
+    return o
+
+
+def masked_block_attn_fwd_v8(q8, q_scale, k8, k_scale, v8, v_scale, block_mask, softmax_scale: float = 0.0,
+                             with_lse: bool = False, workspace=None, out=None, lse=None,
+                             out_dtype=torch.bfloat16, stream=None):
+    """The mask entry on an INT8 V (C ABI ``masked_block_attn_fwd_v8``)."""
+    B, H, _, d = q8.shape
+    Lk = k8.shape[2]
+    _need(v8, torch.int8, (B, H, Lk, d), "v8")
+    _need(v_scale, torch.float32, (B, H, -(-Lk // 64)), "v_scale")
+    return _masked_call("masked_block_attn_fwd_v8", q8, q_scale, k8, k_scale, (v8, v_scale), v8, block_mask,
+                        softmax_scale, with_lse, workspace, out, lse, out_dtype, stream)
 
 
 def check_status(workspace: torch.Tensor, stream=None):

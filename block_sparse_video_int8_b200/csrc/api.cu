@@ -122,7 +122,8 @@ int check_workspace(void* ws, size_t bytes, size_t need) {
 int run_attention(const bsva_shape& s, const int8_t* q8, const float* q_scale, const int8_t* k8,
                   const float* k_scale, const void* v, const uint8_t* kept_mask, const int32_t* kept_idx,
                   const int32_t* kept_cnt, int centroid_mode, float softmax_scale, int out_dtype, void* out,
-                  float* lse, unsigned char* ws, const WsLayout& L, cudaStream_t st) {
+                  float* lse, unsigned char* ws, const WsLayout& L, cudaStream_t st,
+                  const float* v_scale = nullptr) {
   int rc = get_encoder();
   if (rc) return rc;
   const uint64_t BH = uint64_t(s.B) * s.H;
@@ -130,9 +131,14 @@ int run_attention(const bsva_shape& s, const int8_t* q8, const float* q_scale, c
   const CUtensorMapSwizzle swq = s.d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   if ((rc = encode_map(&maps.q8, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.d, s.Lq, BH, s.d, QB, swq, "q8"))) return rc;
   if ((rc = encode_map(&maps.k8, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.d, s.Lk, BH, s.d, KB, swq, "k8"))) return rc;
-  if ((rc = encode_map(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, s.d, s.Lk, BH, 64, KB,
-                       CU_TENSOR_MAP_SWIZZLE_128B, "v")))
+  if (v_scale) {   // INT8 V: whole rows of d bytes, widened in shared memory by the kernel
+    if ((rc = encode_map(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.d, s.Lk, BH, s.d, KB,
+                         CU_TENSOR_MAP_SWIZZLE_NONE, "v8")))
+      return rc;
+  } else if ((rc = encode_map(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, s.d, s.Lk, BH, 64, KB,
+                              CU_TENSOR_MAP_SWIZZLE_128B, "v"))) {
     return rc;
+  }
   if (centroid_mode > 0) {
     const uint64_t nCR = uint64_t(L.nCT) * 64;
     if ((rc = encode_map(&maps.ck8, ws + L.ck8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.d, nCR, BH, s.d, KB, swq, "ck8")))
@@ -157,6 +163,7 @@ int run_attention(const bsva_shape& s, const int8_t* q8, const float* q_scale, c
   a.kept_idx = kept_idx;
   a.kept_cnt = kept_cnt;
   a.kept_mask = kept_mask;
+  a.v_scale = v_scale;
   a.cfac = centroid_mode > 0 ? reinterpret_cast<const float*>(ws + L.cfac) : nullptr;
   a.cbias = centroid_mode > 0 ? reinterpret_cast<const float*>(ws + L.cbias) : nullptr;
   a.order = nullptr;
@@ -391,6 +398,46 @@ int masked_block_attn_fwd(bsva_shape s, const int8_t* q8, const float* q_scale, 
   if (e != cudaSuccess) return cuda_fail(e, "mask expansion launch");
   return run_attention(s, q8, q_scale, k8, k_scale, v, nullptr, kidx, kcnt, 0, softmax_scale, out_dtype, out, lse,
                        ws, L, st);
+}
+
+int bsva_quantize_v(bsva_shape s, const void* v, int8_t* v8, float* v_scale, bsva_stream_t stream) {
+  int rc;
+  if ((rc = check_shape(s))) return rc;
+  REQUIRE_PTR(v, 16); REQUIRE_PTR(v8, 16); REQUIRE_PTR(v_scale, 4);
+  if ((rc = check_device())) return rc;
+  cudaError_t e = launch_quant_v(s, reinterpret_cast<const __nv_bfloat16*>(v), v8, v_scale,
+                                 reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "V quantiser launch");
+  return ok();
+}
+
+int masked_block_attn_fwd_v8(bsva_shape s, const int8_t* q8, const float* q_scale, const int8_t* k8,
+                             const float* k_scale, const int8_t* v8, const float* v_scale,
+                             const uint8_t* block_mask, int mask_heads, float softmax_scale, int out_dtype,
+                             void* out, float* lse, void* workspace, size_t workspace_bytes,
+                             bsva_stream_t stream) {
+  int rc;
+  if ((rc = check_shape(s))) return rc;
+  if (mask_heads != 1 && mask_heads != s.H)
+    return fail(BSVA_ERR_INVALID_ARG, "mask_heads = %d must be 1 or H = %d", mask_heads, s.H);
+  if (std::isnan(softmax_scale) || std::isinf(softmax_scale))
+    return fail(BSVA_ERR_INVALID_ARG, "softmax_scale must be finite");
+  if (out_dtype != BSVA_OUT_BF16 && out_dtype != BSVA_OUT_F32)
+    return fail(BSVA_ERR_INVALID_ARG, "out_dtype = %d; use BSVA_OUT_BF16 (0) or BSVA_OUT_F32 (1)", out_dtype);
+  REQUIRE_PTR(q8, 16); REQUIRE_PTR(q_scale, 4); REQUIRE_PTR(k8, 16); REQUIRE_PTR(k_scale, 4);
+  REQUIRE_PTR(v8, 16); REQUIRE_PTR(v_scale, 4); REQUIRE_PTR(block_mask, 1); REQUIRE_PTR(out, 16);
+  if (lse && !aligned(lse, 4)) return fail(BSVA_ERR_INVALID_ARG, "lse is not 4-byte aligned");
+  const WsLayout L = ws_layout(s, 0);
+  if ((rc = check_workspace(workspace, workspace_bytes, L.total))) return rc;
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  int32_t* kidx = reinterpret_cast<int32_t*>(ws + L.kidx);
+  int32_t* kcnt = reinterpret_cast<int32_t*>(ws + L.kcnt);
+  cudaError_t e = launch_mask_expand(s, block_mask, mask_heads, kidx, kcnt, st);
+  if (e != cudaSuccess) return cuda_fail(e, "mask expansion launch");
+  return run_attention(s, q8, q_scale, k8, k_scale, v8, nullptr, kidx, kcnt, 0, softmax_scale, out_dtype, out, lse,
+                       ws, L, st, v_scale);
 }
 
 int bsva_check_status(void* workspace, bsva_stream_t stream) {

@@ -24,6 +24,13 @@
 //              accumulate) and O += P . V with kind::f16 (A = P from TMEM,
 //              B = V from shared memory, fp32 accumulate). S is double
 //              buffered so QK of tile n+1 overlaps the softmax of tile n.
+// INT8 V (mask entry; "FlashVSR Kitchen Sparse Attention", intro: the
+// streaming cache keeps K/V as INT8 and the kernel eats it without rebuilding
+// bf16 tensors): the V tile lands in the upper half of its bf16 stage and the
+// MMA warp widens it in place to bf16 integers (exact, |v8| <= 127) before
+// its PV; the block scale s_j is folded into the exponent, P' = 2^(y + log2 s_j),
+// and the row sums take the rounded P' times 1/s_j, so numerator and
+// denominator weight each key alike.
 // Centroid tiles hold 32 groups as (hi, lo) INT8 row pairs (pool = 128 hi + lo)
 // so their dot with q8 is exact in int32; the value rows are (bf16 hi, bf16 lo)
 // and share one probability.
@@ -51,7 +58,7 @@ struct TileMeta {
   float f;          // kept tiles: sq*sk*scale*log2e
   int nvalid;       // kept tiles: valid key columns (64 except a tail block)
   int centroid;     // 1 = centroid tile
-  int pad;
+  float vlog2;      // INT8 V: log2 of the V block scale (0 for a zero block); unused for bf16 V
 };
 
 template <int D>
@@ -85,7 +92,8 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-template <int D>
+// kV8: V is INT8 with per-block scales (a.v_scale), P and V enter PV as f16.
+template <int D, bool kV8>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_kernel(const AttnArgs a, const __grid_constant__ AttnMaps maps) {
   extern __shared__ unsigned char smem_raw[];
@@ -197,6 +205,10 @@ __global__ void __launch_bounds__(kThreads, 2)
           mt.f = f_next;
           mt.nvalid = min(KB, a.Lk - row);
           mt.centroid = 0;
+          if constexpr (kV8) {
+            const float sv = a.v_scale[size_t(bh) * a.nKB + j_next];
+            mt.vlog2 = sv > 0.f ? __log2f(sv) : 0.f;
+          }
         }
       } else {
         const int tc = t - n_exact;
@@ -227,7 +239,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     // 1 KB, the two 64-column halves (D = 128) 8 KB apart.
     constexpr uint32_t kLboV = KB * 128, kSboV = 1024;
     constexpr uint32_t IDESC_QK = make_idesc(2, 1, 1, false, false, 128, 64);
-    constexpr uint32_t IDESC_PV = make_idesc(1, 1, 1, false, true, 128, D);
+    constexpr uint32_t kFmtPV = kV8 ? 0u : 1u;   // f16 (INT8 V widened) or bf16
+    constexpr uint32_t IDESC_PV = make_idesc(1, kFmtPV, kFmtPV, false, true, 128, D);
     constexpr uint32_t kStrideK = (KB * D) >> 4, kStrideV = (KB * D * 2) >> 4;   // stage strides, 16 B units
     const uint64_t dq = make_sdesc(smem_u32(sm.q), 16, kSboQK, kLayoutQK);
     const uint64_t dk0 = make_sdesc(smem_u32(sm.k[0]), 16, kSboQK, kLayoutQK);
@@ -270,11 +283,57 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (t >= NV && !wait(&sm.v_empty[sv], ((t / NV) - 1) & 1)) return false;
       if (lane == 0) {
         const int row = sm.vrow[t % NR];
-        const CUtensorMap* mv = t < n_exact ? &maps.v : &maps.cv;
-        mbar_arrive_expect_tx(&sm.v_full[sv], KB * D * 2);
-        tma_load_3d(sm.v[sv], mv, 0, row, bh, &sm.v_full[sv]);
-        if (D == 128) tma_load_3d(sm.v[sv] + KB * 64, mv, 64, row, bh, &sm.v_full[sv]);
+        if constexpr (kV8) {
+          // INT8 rows of D bytes into the upper half of the stage; widened before its PV
+          mbar_arrive_expect_tx(&sm.v_full[sv], KB * D);
+          tma_load_3d(reinterpret_cast<unsigned char*>(sm.v[sv]) + KB * D, &maps.v, 0, row, bh, &sm.v_full[sv]);
+        } else {
+          const CUtensorMap* mv = t < n_exact ? &maps.v : &maps.cv;
+          mbar_arrive_expect_tx(&sm.v_full[sv], KB * D * 2);
+          tma_load_3d(sm.v[sv], mv, 0, row, bh, &sm.v_full[sv]);
+          if (D == 128) tma_load_3d(sm.v[sv] + KB * 64, mv, 64, row, bh, &sm.v_full[sv]);
+        }
       }
+      __syncwarp();
+      return true;
+    };
+    // INT8 V: widen tile t in place to the f16 layout PV reads (MN-major rows of 64 values,
+    // 128 bytes, 128-byte swizzle; the two 64-column halves 8 KB apart). Every INT8 byte is
+    // read into registers before the first store, since the f16 tile overwrites them.
+    // x in [-127, 127] -> f16 bits 0x6400 | (x + 128) = 1024 + x + 128, minus 1152: exact.
+    auto v_widen = [&](int t) -> bool {
+      const int sv = t % NV;
+      if (!wait(&sm.v_full[sv], (t / NV) & 1)) return false;
+      unsigned char* stage = reinterpret_cast<unsigned char*>(sm.v[sv]);
+      const unsigned char* src = stage + KB * D;
+      constexpr int CPR = D / 16;              // 16-byte INT8 chunks per row
+      constexpr int NCH = KB * CPR / 32;       // chunks per lane
+      uint4 in[NCH];
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) in[i] = *reinterpret_cast<const uint4*>(src + (lane + 32 * i) * 16);
+      __syncwarp();
+      const __half2 k1152 = __floats2half2_rn(1152.f, 1152.f);
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) {
+        const int q = lane + 32 * i;
+        const int r = q / CPR, c16 = q % CPR;   // key row; INT8 columns 16*c16 .. 16*c16+15
+        const int j0 = (2 * c16) % 8;           // first 16-byte f16 chunk in the half's row
+        unsigned char* rowp = stage + ((16 * c16) / 64) * (KB * 128) + r * 128;
+        const uint32_t w[4] = {in[i].x ^ 0x80808080u, in[i].y ^ 0x80808080u, in[i].z ^ 0x80808080u,
+                               in[i].w ^ 0x80808080u};
+        uint32_t o[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          uint32_t lo = __byte_perm(w[e], 0x64646464u, 0x5140), hi = __byte_perm(w[e], 0x64646464u, 0x5342);
+          __half2 hl = __hsub2(*reinterpret_cast<__half2*>(&lo), k1152);
+          __half2 hh = __hsub2(*reinterpret_cast<__half2*>(&hi), k1152);
+          o[2 * e] = *reinterpret_cast<uint32_t*>(&hl);
+          o[2 * e + 1] = *reinterpret_cast<uint32_t*>(&hh);
+        }
+        *reinterpret_cast<uint4*>(rowp + ((j0 ^ (r & 7)) * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(rowp + (((j0 + 1) ^ (r & 7)) * 16)) = make_uint4(o[4], o[5], o[6], o[7]);
+      }
+      fence_proxy_async_smem();   // the tensor core reads the widened tile
       __syncwarp();
       return true;
     };
@@ -288,6 +347,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (ok) { tc_fence_after(); do_qk(n); }
       if (ok) ok = v_load(n);
     }
+    if constexpr (kV8) {
+      if (ok) ok = v_widen(0);
+    }
     for (int n = 0; ok && n < N; ++n) {
       ok = wait(&sm.p_full[n & 1], (n >> 1) & 1) && wait(&sm.v_full[n % NV], (n / NV) & 1);
       if (!ok) break;
@@ -300,6 +362,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         // tile arrives by TMA under its own barrier
         if (ok) do_qk(n + 2);
         if (ok) ok = v_load(n + 2);   // needs PV(n - 1), issued one step ago
+      }
+      if constexpr (kV8) {
+        if (ok && n + 1 < N) ok = v_widen(n + 1);   // while the softmax works on tile n + 1
       }
     }
     if (elect_one()) tc_commit(&sm.o_full);
@@ -372,19 +437,35 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         // P = 2^(x*f - m) as bf16 pairs; lsum adds the bf16-rounded weights
         // the PV product uses, esum the unrounded ones (log-sum-exp only).
+        // INT8 V: the weights carry the V block scale, P' = 2^(y + log2 s_j), and the sums
+        // take P' * 2^-(log2 s_j), so both sides of O / l see the same (rounded) weights.
+        const float vlog2 = kV8 ? mt.vlog2 : 0.f;
+        const float vinv = kV8 ? ex2(-vlog2) : 1.f;
         auto exps = [&](float m_use) {
-          const float2 f2 = make_float2(f, f), nm2 = make_float2(-m_use, -m_use);
+          const float2 f2 = make_float2(f, f);
+          const float nm = kV8 ? vlog2 - m_use : -m_use;
+          const float2 nm2 = make_float2(nm, nm);
           float2 la = make_float2(0.f, 0.f), ea = make_float2(0.f, 0.f);
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const float2 y = __ffma2_rn(make_float2(xs[2 * c], xs[2 * c + 1]), f2, nm2);
             const float p0 = ex2(y.x), p1 = ex2(y.y);
-            pk[c] = pack_bf16x2(p0, p1);
-            la = __fadd2_rn(la, make_float2(__uint_as_float(pk[c] << 16), __uint_as_float(pk[c] & 0xFFFF0000u)));
+            if constexpr (kV8) {
+              pk[c] = pack_f16x2(p0, p1);
+              const __half2 h = *reinterpret_cast<const __half2*>(&pk[c]);
+              la = __fadd2_rn(la, __half22float2(h));
+            } else {
+              pk[c] = pack_bf16x2(p0, p1);
+              la = __fadd2_rn(la, make_float2(__uint_as_float(pk[c] << 16), __uint_as_float(pk[c] & 0xFFFF0000u)));
+            }
             if (want_lse) ea = __fadd2_rn(ea, make_float2(p0, p1));
           }
           lsum = la.x + la.y;
           esum = ea.x + ea.y;
+          if constexpr (kV8) {
+            lsum *= vinv;
+            esum *= vinv;
+          }
         };
         // Speculate that the running max still holds (it nearly always does
         // after the first tiles), so the exps need not wait for this tile's max.
@@ -512,16 +593,21 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-template <int D>
-cudaError_t launch_attn_d(const AttnArgs& a, const AttnMaps& maps, cudaStream_t st) {
+template <int D, bool kV8>
+cudaError_t launch_attn_dv(const AttnArgs& a, const AttnMaps& maps, cudaStream_t st) {
   // At least 100 KB so that no more than two CTAs share an SM: two 256-column
   // TMEM allocations fill the SM's 512 columns.
   const size_t smem = sizeof(Smem<D>) + 1024 > 100 * 1024 ? sizeof(Smem<D>) + 1024 : 100 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, kV8>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   const unsigned grid = unsigned(a.B) * a.H * a.nQB;
-  attn_kernel<D><<<grid, kThreads, smem, st>>>(a, maps);
+  attn_kernel<D, kV8><<<grid, kThreads, smem, st>>>(a, maps);
   return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_attn_d(const AttnArgs& a, const AttnMaps& maps, cudaStream_t st) {
+  return a.v_scale ? launch_attn_dv<D, true>(a, maps, st) : launch_attn_dv<D, false>(a, maps, st);
 }
 
 // One CTA waits on a barrier nothing arrives at; the bounded wait runs out.

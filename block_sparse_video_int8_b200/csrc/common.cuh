@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "bsva.h"
 
@@ -305,6 +306,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));   // first source -> upper half
+  return r;
+}
+
+// Generic-proxy shared-memory stores become visible to the async proxy (tensor core, TMA).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 }  // namespace bsva
 
 // ------------------------------------------------------- host-side launchers --
@@ -322,6 +334,7 @@ struct AttnArgs {
   const int32_t* kept_idx;  // [BH, nQB, nKB]
   const int32_t* kept_cnt;  // [BH, nQB]
   const uint8_t* kept_mask; // [BH, nQB, nKB] (centroid exclusion), may be null when mode 0
+  const float* v_scale;     // [BH, nKB] per-block scales of an INT8 V (mask entry), null for bf16 V
   const float* cfac;        // [BH, nCT*32]
   const float* cbias;       // [BH, nCT*32]
   const int32_t* order;     // [BH*nQB] work order
@@ -339,6 +352,8 @@ struct AttnMaps {
 cudaError_t launch_quant_pool(const bsva_shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, int8_t* q8,
                               float* q_scale, int8_t* k8, float* k_scale, int32_t* q_pool, int32_t* k_pool,
                               cudaStream_t st);
+// The K quantiser alone over another [B, H, Lk, d] tensor (INT8 V), no pools.
+cudaError_t launch_quant_v(const bsva_shape& s, const __nv_bfloat16* v, int8_t* v8, float* v_scale, cudaStream_t st);
 cudaError_t launch_route(const bsva_shape& s, double tau, const int32_t* q_pool, const int32_t* k_pool,
                          const float* k_scale, double* scores, uint8_t* kept_mask, int32_t* kept_idx,
                          int32_t* kept_cnt, double* row_stats, cudaStream_t st);

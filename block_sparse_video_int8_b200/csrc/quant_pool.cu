@@ -51,13 +51,13 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, BSVA_QP_MINB) quant_pool_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, int8_t* __restrict__ q8,
     float* __restrict__ q_scale, int8_t* __restrict__ k8, float* __restrict__ k_scale,
-    int32_t* __restrict__ q_pool, int32_t* __restrict__ k_pool, int Lq, int Lk) {
+    int32_t* __restrict__ q_pool, int32_t* __restrict__ k_pool, int Lq, int Lk, int z0) {
   constexpr int CPR = D / 8;                 // 16-byte chunks per row
   constexpr int NC = QB * CPR / kThreads;    // chunks per thread (8 for d=128)
   constexpr int RSTEP = kThreads / CPR;      // row step between a thread's chunks
   constexpr int CPQ = 32 / RSTEP;            // chunks per 32-row quarter
   static_assert(RSTEP <= 32 && 32 % RSTEP == 0 && NC == 4 * CPQ, "slab tiling");
-  const bool isK = blockIdx.z == 1;
+  const bool isK = blockIdx.z + z0 == 1;   // z0 = 1: K part only (the INT8 V entry)
   const int L = isK ? Lk : Lq;
   const int slab = blockIdx.x;
   const int r0 = slab * QB;
@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, BSVA_QP_MINB) quant_pool_kernel(
       for (int r = 0; r < RSTEP; ++r) tot += s_red[(hq * RSTEP + r) * D + rem];
       const int col = 8 * ((rem / 4) % CPR) + 4 * (rem / (4 * CPR)) + (rem % 4);
       const int kb = 2 * slab + (hq >> 1);
-      if (kb < nKB) k_pool[((size_t(bh) * nKB + kb) * 2 + (hq & 1)) * D + col] = __float2int_rn(tot);
+      if (kb < nKB && k_pool) k_pool[((size_t(bh) * nKB + kb) * 2 + (hq & 1)) * D + col] = __float2int_rn(tot);
     }
     if (t < 2) {
       const int kb = 2 * slab + t;
@@ -199,10 +199,21 @@ cudaError_t launch_quant_pool(const bsva_shape& s, const __nv_bfloat16* q, const
   const int slabs = (max(s.Lq, s.Lk) + QB - 1) / QB;
   dim3 grid(slabs, s.B * s.H, 2);
   if (s.d == 128) {
-    quant_pool_kernel<128><<<grid, kThreads, 0, st>>>(q, k, q8, q_scale, k8, k_scale, q_pool, k_pool, s.Lq, s.Lk);
+    quant_pool_kernel<128><<<grid, kThreads, 0, st>>>(q, k, q8, q_scale, k8, k_scale, q_pool, k_pool, s.Lq, s.Lk, 0);
   } else {
-    quant_pool_kernel<64><<<grid, kThreads, 0, st>>>(q, k, q8, q_scale, k8, k_scale, q_pool, k_pool, s.Lq, s.Lk);
+    quant_pool_kernel<64><<<grid, kThreads, 0, st>>>(q, k, q8, q_scale, k8, k_scale, q_pool, k_pool, s.Lq, s.Lk, 0);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_v(const bsva_shape& s, const __nv_bfloat16* v, int8_t* v8, float* v_scale, cudaStream_t st) {
+  dim3 grid((s.Lk + QB - 1) / QB, s.B * s.H, 1);
+  if (s.d == 128)
+    quant_pool_kernel<128><<<grid, kThreads, 0, st>>>(nullptr, v, nullptr, nullptr, v8, v_scale, nullptr, nullptr,
+                                                      s.Lq, s.Lk, 1);
+  else
+    quant_pool_kernel<64><<<grid, kThreads, 0, st>>>(nullptr, v, nullptr, nullptr, v8, v_scale, nullptr, nullptr,
+                                                     s.Lq, s.Lk, 1);
   return cudaGetLastError();
 }
 

@@ -229,6 +229,32 @@ int masked_block_attn_fwd(bsva_shape s, const int8_t* q8, const float* q_scale,
                           size_t workspace_bytes,
                           bsva_stream_t stream);
 
+/* Per-block symmetric INT8 quantisation of V with the K quantiser (64-row
+ * blocks, s = fl32(amax/127), x8 = rint_half_even(fl32(x/s))), the format of
+ * an INT8 K/V cache ("FlashVSR Kitchen Sparse Attention", intro: the
+ * streaming cache keeps K and V as INT8).
+ *   v        bf16 [B,H,Lk,d]
+ *   v8       out: int8 [B,H,Lk,d]
+ *   v_scale  out: fp32 [B,H,nKB]                                             */
+int bsva_quantize_v(bsva_shape s, const void* v, int8_t* v8, float* v_scale,
+                    bsva_stream_t stream);
+
+/* masked_block_attn_fwd on an INT8 V ("FlashVSR Kitchen Sparse Attention",
+ * intro: the INT8 cache is fed straight to the kernel, with no
+ * full-precision rebuild of K and V). The output is softmax attention over
+ * the dequantised values v8 * v_scale[block]; in the kernel the block scale
+ * rides in the weights, P' = P * s_j, the INT8 tile is widened to f16 in
+ * shared memory (exact), and PV runs as f16 x f16 with fp32 accumulation.
+ *   v8, v_scale  as written by bsva_quantize_v
+ *   Every other argument as in masked_block_attn_fwd.                        */
+int masked_block_attn_fwd_v8(bsva_shape s, const int8_t* q8, const float* q_scale,
+                             const int8_t* k8, const float* k_scale,
+                             const int8_t* v8, const float* v_scale,
+                             const uint8_t* block_mask, int mask_heads,
+                             float softmax_scale, int out_dtype, void* out,
+                             float* lse, void* workspace, size_t workspace_bytes,
+                             bsva_stream_t stream);
+
 /* masked_block_attn_fwd without a workspace. The source pages have no
  * counterpart: this entry point is for callers that cannot allocate device
  * memory, such as a plugin inside a host application whose allocator already

@@ -202,3 +202,38 @@ def topk_parity(bsva, w, sparsity, heads=None, q_blocks=None, centroid_mode=None
                                                    keep, mode, 0.0, q_blocks=blocks)
         compare_rows(to_np(out[b, h].float()), to_np(lse[b, h]), O_ref, lse_ref, q_rows(w.Lq, blocks), rep)
     return route, out, lse, rep
+
+
+def masked_parity_v8(bsva, w, mask, heads=None, q_blocks=None, softmax_scale=0.0, V=None):
+    """The mask entry on INT8 V: the GPU quantises V and runs the entry; the oracle
+    quantises V with its own quantiser (checked bit for bit) and attends over the
+    dequantised values."""
+    Q, K, V0 = inputs(w)
+    V = V0 if V is None else V.to("cuda")
+    qk = bsva.quantize_qk(Q, K)
+    vq = bsva.quantize_v(V)
+    m_dev = mask.to("cuda")
+    out, lse = bsva.masked_block_attn_fwd_v8(qk["q8"], qk["q_scale"], qk["k8"], qk["k_scale"], vq["v8"],
+                                             vq["v_scale"], m_dev, softmax_scale=softmax_scale, with_lse=True,
+                                             out_dtype=torch.float32)
+    out16 = bsva.masked_block_attn_fwd_v8(qk["q8"], qk["q_scale"], qk["k8"], qk["k_scale"], vq["v8"],
+                                          vq["v_scale"], m_dev, softmax_scale=softmax_scale)
+    torch.cuda.synchronize()
+    assert torch.equal(out16, out.to(torch.bfloat16)), "bf16 output != round(fp32 output)"
+    heads = heads or [(b, h) for b in range(w.B) for h in range(w.H)]
+    rep = Report()
+    Hm = mask.shape[1]
+    for b, h in heads:
+        q, k, _ = head_np(w, b, h)
+        v = V[b, h].float().cpu().numpy()
+        ref = oracle.route_head(q, k, -math.inf, 0)
+        v8, sv = oracle.quantize_blocks(v, 64)
+        assert np.array_equal(to_np(vq["v8"][b, h]), v8), "v8 differs"
+        assert np.array_equal(to_np(vq["v_scale"][b, h]), sv), "v_scale differs"
+        vdeq = oracle.dequantize_blocks(v8, sv, 64)
+        allowed = oracle.physical_allowed(mask[b, h % Hm].numpy(), w.nKB)
+        blocks = list(range(w.nQB)) if q_blocks is None else [i for i in q_blocks if i < w.nQB]
+        O_ref, lse_ref = oracle.masked_attention_head(ref["q8"], ref["q_scale"], ref["k8"], ref["k_scale"], vdeq,
+                                                      allowed, softmax_scale, q_blocks=blocks)
+        compare_rows(to_np(out[b, h].float()), to_np(lse[b, h]), O_ref, lse_ref, q_rows(w.Lq, blocks), rep)
+    return out, lse, rep

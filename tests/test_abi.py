@@ -108,6 +108,21 @@ def test_lcsa_builder_rejects_bad_geometry():
     assert lib.bsva_build_lcsa_mask(100, 100, 64, 1, 1, None, None) == 1
 
 
+def test_int8_v_entries_reject_bad_arguments():
+    lib = bsva.load()
+    s = bsva.Shape(1, 2, 256, 256, 128, 0)
+    P = ctypes.c_void_p(0x10000)
+    assert lib.bsva_quantize_v(s, P, None, P, None) == 1
+    assert lib.bsva_quantize_v(bsva.Shape(1, 2, 256, 256, 96, 0), P, P, P, None) == 2
+    rc = lib.masked_block_attn_fwd_v8(s, P, P, P, P, None, P, P, 1, ctypes.c_float(0), 0, P, None, P, 1 << 30,
+                                      None)
+    assert rc == 1 and b"v8" in lib.bsva_last_error()
+    rc = lib.masked_block_attn_fwd_v8(s, P, P, P, P, P, P, P, 3, ctypes.c_float(0), 0, P, None, P, 1 << 30, None)
+    assert rc == 1                                                 # mask_heads not in {1, H}
+    rc = lib.masked_block_attn_fwd_v8(s, P, P, P, P, P, P, P, 1, ctypes.c_float(0), 0, P, None, P, 16, None)
+    assert rc == 3
+
+
 def test_fwd_rejects_bad_mode_and_small_workspace():
     lib = bsva.load()
     s = bsva.Shape(1, 2, 256, 256, 128, 0)

@@ -13,8 +13,8 @@ import torch
 
 import oracle
 import workloads
-from parity import (Report, assert_within, compare_rows, head_np, inputs, masked_parity, q_rows,
-                    sol_parity, to_np, topk_parity)
+from parity import (Report, assert_within, compare_rows, head_np, inputs, masked_parity, masked_parity_v8,
+                    q_rows, sol_parity, to_np, topk_parity)
 
 pytestmark = pytest.mark.gpu
 
@@ -99,6 +99,26 @@ def test_masked_small_lcsa_device_mask(gpu_lib):
     assert_within(rep, "lcsa_small device mask")
 
 
+def test_masked_v8_small_lcsa(gpu_lib):
+    w = workloads.get("lcsa_small")
+    _, _, rep = masked_parity_v8(gpu_lib, w, workloads.block_mask(w))
+    assert_within(rep, "lcsa_small INT8 V")
+
+
+@pytest.mark.parametrize("name", ["cross", "ragged_d64"])
+def test_masked_v8_random_mask_zero_block_and_empty_rows(gpu_lib, name):
+    w = workloads.get(name)
+    rng = np.random.default_rng(9)
+    m = (rng.random((w.B, w.H, w.nQB, w.nLK)) < 0.45).astype(np.uint8)
+    m[0, 0, 1, :] = 0                       # a query block with nothing allowed
+    m[0, 0, 0, :] = 1
+    _, _, V = inputs(w)
+    V[0, 0, 64:128] = 0                     # an all-zero V block: scale 0
+    out, lse, rep = masked_parity_v8(gpu_lib, w, torch.from_numpy(m), softmax_scale=0.09, V=V)
+    assert_within(rep, f"{name} INT8 V")
+    assert bool((out[0, 0, 128:256] == 0).all()) and bool(torch.isneginf(lse[0, 0, 128:256]).all())
+
+
 def test_masked_per_head_random_mask_with_empty_rows(gpu_lib):
     w = workloads.get("cross")
     rng = np.random.default_rng(5)
@@ -152,6 +172,15 @@ def _sample_blocks(nQB, n_extra=4, seed=0):
     base = {0, 1, nQB // 2, nQB - 1}
     base |= set(int(x) for x in rng.choice(nQB, size=n_extra, replace=False))
     return sorted(base)
+
+
+@pytest.mark.slow
+def test_full_lcsa_v8(gpu_lib):
+    w = workloads.get("lcsa")
+    heads = [(0, 0), (0, w.H - 1)]
+    _, _, rep = masked_parity_v8(gpu_lib, w, workloads.block_mask(w), heads=heads,
+                                 q_blocks=_sample_blocks(w.nQB))
+    assert_within(rep, "lcsa full INT8 V")
 
 
 @pytest.mark.slow
