@@ -250,11 +250,36 @@ ATTN_SOURCES = ("block_sparse_video_int8_b200/csrc/attn_sm100.cu", "block_sparse
 TRAFFIC_FILE = "profiles/attn_sm100_traffic.md"
 
 
+def _code_only(text: str) -> str:
+    """Source text without comments and whitespace runs (string literals kept):
+    the traffic figure stays valid across comment-only edits."""
+    import re
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"':                                   # string literal, copied as is
+            j = i + 1
+            while j < n and text[j] != '"':
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            i = text.find("\n", i)
+            i = n if i < 0 else i
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return re.sub(r"\s+", " ", "".join(out)).strip()
+
+
 def attn_source_hash() -> str:
     import hashlib
     h = hashlib.sha256()
     for f in ATTN_SOURCES:
-        h.update(open(os.path.join(ROOT, f), "rb").read())
+        h.update(_code_only(open(os.path.join(ROOT, f), encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 

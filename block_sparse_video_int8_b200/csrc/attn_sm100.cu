@@ -26,10 +26,11 @@
 //              buffered so QK of tile n+1 overlaps the softmax of tile n.
 // INT8 V (mask entry; "FlashVSR Kitchen Sparse Attention", intro: the
 // streaming cache keeps K/V as INT8 and the kernel eats it without rebuilding
-// bf16 tensors): the V tile lands in the upper half of its bf16 stage and the
-// MMA warp widens it in place to bf16 integers (exact, |v8| <= 127) before
-// its PV; the block scale s_j is folded into the exponent, P' = 2^(y + log2 s_j),
-// and the row sums take the rounded P' times 1/s_j, so numerator and
+// bf16 tensors; the kV8 instantiation): the V tile lands in the upper half of
+// its stage and the MMA warp widens it in place to f16 integers (exact,
+// |v8| <= 127) before its PV, which then runs as f16 x f16 with P packed as
+// f16; the block scale s_j is folded into the exponent, P' = 2^(y + log2 s_j),
+// and the row sums take the rounded P' times 2^-log2 s_j, so numerator and
 // denominator weight each key alike.
 // Centroid tiles hold 32 groups as (hi, lo) INT8 row pairs (pool = 128 hi + lo)
 // so their dot with q8 is exact in int32; the value rows are (bf16 hi, bf16 lo)

@@ -50,3 +50,13 @@ def test_two_rank_max_and_barrier():
 def test_single_rank_is_identity():
     import bench
     assert bench._max_over_ranks(None, 2.5) == 2.5
+
+
+def test_traffic_hash_ignores_comments_but_not_code():
+    import bench
+    a = 'int a; // note\n/* block */ asm("x // y"); int  b;\n'
+    b = 'int a;\n asm("x // y");    int b; // another note\n'
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(a) != bench._code_only(a.replace("int  b", "int c"))
+    assert bench._code_only(a) != bench._code_only(a.replace("x // y", "x / y"))   # strings are code
+    assert bench.measured_traffic("wan14b") is not None        # the committed profile matches the sources
