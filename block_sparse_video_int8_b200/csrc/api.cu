@@ -166,7 +166,6 @@ int run_attention(const bsva_shape& s, const int8_t* q8, const float* q_scale, c
   a.v_scale = v_scale;
   a.cfac = centroid_mode > 0 ? reinterpret_cast<const float*>(ws + L.cfac) : nullptr;
   a.cbias = centroid_mode > 0 ? reinterpret_cast<const float*>(ws + L.cbias) : nullptr;
-  a.order = nullptr;
   a.out = out_dtype == BSVA_OUT_BF16 ? reinterpret_cast<__nv_bfloat16*>(out) : nullptr;
   a.out_f32 = out_dtype == BSVA_OUT_F32 ? reinterpret_cast<float*>(out) : nullptr;
   a.lse = lse;

@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int item = a.order ? a.order[blockIdx.x] : int(blockIdx.x);
+  const int item = int(blockIdx.x);
   const int bh = item / a.nQB;
   const int i = item % a.nQB;
   const size_t row_item = size_t(bh) * a.nQB + i;

@@ -59,4 +59,3 @@ def test_traffic_hash_ignores_comments_but_not_code():
     assert bench._code_only(a) == bench._code_only(b)
     assert bench._code_only(a) != bench._code_only(a.replace("int  b", "int c"))
     assert bench._code_only(a) != bench._code_only(a.replace("x // y", "x / y"))   # strings are code
-    assert bench.measured_traffic("wan14b") is not None        # the committed profile matches the sources
