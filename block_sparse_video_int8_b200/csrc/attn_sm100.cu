@@ -279,9 +279,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     auto wait = [&](uint64_t* bar, uint32_t par) { return __all_sync(0xffffffffu, mbar_wait(bar, par, abort, a.status, lim)); };
     // V(t) into stage t % NV once PV(t - NV) has landed; its row was published
     // with K(t)'s barrier, which this warp has already waited on.
-    auto v_load = [&](int t) -> bool {
+    auto v_load = [&](int t, bool stage_free) -> bool {
       const int sv = t % NV;
-      if (t >= NV && !wait(&sm.v_empty[sv], ((t / NV) - 1) & 1)) return false;
+      if (t >= NV && !stage_free && !wait(&sm.v_empty[sv], ((t / NV) - 1) & 1)) return false;
       if (lane == 0) {
         const int row = sm.vrow[t % NR];
         if constexpr (kV8) {
@@ -346,23 +346,30 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int n = 0; ok && n < 2 && n < N; ++n) {
       ok = wait(&sm.k_full[n % NK], (n / NK) & 1);
       if (ok) { tc_fence_after(); do_qk(n); }
-      if (ok) ok = v_load(n);
+      if (ok) ok = v_load(n, true);
     }
     if constexpr (kV8) {
       if (ok) ok = v_widen(0);
     }
     for (int n = 0; ok && n < N; ++n) {
-      ok = wait(&sm.p_full[n & 1], (n >> 1) & 1) && wait(&sm.v_full[n % NV], (n / NV) & 1);
+      // The barriers of this step that are usually complete already are tested
+      // together, so their round trips overlap instead of adding up.
+      const bool v_in = mbar_test_wait(&sm.v_full[n % NV], (n / NV) & 1);
+      const bool k_in = n + 2 >= N || mbar_test_wait(&sm.k_full[(n + 2) % NK], ((n + 2) / NK) & 1);
+      const bool e_in = n + 2 >= N || n + 2 < NV ||
+                        mbar_test_wait(&sm.v_empty[(n + 2) % NV], (((n + 2) / NV) - 1) & 1);
+      ok = wait(&sm.p_full[n & 1], (n >> 1) & 1) &&
+           (__all_sync(0xffffffffu, v_in) || wait(&sm.v_full[n % NV], (n / NV) & 1));
       if (!ok) break;
       tc_fence_after();
       do_pv(n);
       if (n + 2 < N) {
-        ok = wait(&sm.k_full[(n + 2) % NK], ((n + 2) / NK) & 1);
+        ok = __all_sync(0xffffffffu, k_in) || wait(&sm.k_full[(n + 2) % NK], ((n + 2) / NK) & 1);
         // no second fence: the one after the p_full wait above already orders this
         // QK's S writes after the softmax warps' loads of that buffer, and the K
         // tile arrives by TMA under its own barrier
         if (ok) do_qk(n + 2);
-        if (ok) ok = v_load(n + 2);   // needs PV(n - 1), issued one step ago
+        if (ok) ok = v_load(n + 2, __all_sync(0xffffffffu, e_in));   // needs PV(n - 1), issued one step ago
       }
       if constexpr (kV8) {
         if (ok && n + 1 < N) ok = v_widen(n + 1);   // while the softmax works on tile n + 1
@@ -401,9 +408,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int n = 0; n < N; ++n) {
       n_cur = n;
       const int sk = n % NK;
+      // the tile's metadata is published with its K stage's barrier (long complete once S
+      // is in); testing it first overlaps the two round trips
+      const bool meta_in = mbar_test_wait(&sm.k_full[sk], (n / NK) & 1);
       bool ok = mbar_wait(&sm.s_full[n & 1], (n >> 1) & 1, abort, a.status, lim);
-      // the tile's metadata is published with its K stage's barrier (long complete once S is in)
-      ok = ok && mbar_wait(&sm.k_full[sk], (n / NK) & 1, abort, a.status, lim);
+      ok = ok && (meta_in || mbar_wait(&sm.k_full[sk], (n / NK) & 1, abort, a.status, lim));
       if (!__all_sync(0xffffffffu, ok)) {
         alive = false;
         break;
