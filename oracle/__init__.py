@@ -22,7 +22,10 @@ What it computes, step by step, and where the source pages describe it:
 * ``attention`` softmax attention over the kept blocks exactly plus one
                 centroid term per skipped 64-token block (1x64) or two 32-token
                 centroids (2x32); and the explicit logical-block-mask entry
-                (LCSA, "FlashVSR Sparge Attention", intro and *How it works*).
+                (LCSA, "FlashVSR Sparge Attention", intro and *How it works*);
+                the residual virtual K/V mode, physical keys exact and each
+                added virtual slice as centroid terms ("Configure H3 Static
+                Virtual KV").
 
 Every function is pinned by ``tests/test_oracle_*.py`` against something
 other than itself (brute force, closed forms, dense softmax attention through
@@ -34,11 +37,11 @@ from .quant import quantize_blocks, dequantize_blocks, q_pools, k_half_pools, bl
 from .route import proxy_scores, sol_route, route_head, topk_keep_count, topk_route
 from .attention import (centroid_groups, centroid_table, sol_attention_head,
                         masked_attention_head, physical_allowed, lcsa_mask,
-                        resolve_scale)
+                        resolve_scale, virtual_kv_residual_head)
 
 __all__ = [
     "quantize_blocks", "dequantize_blocks", "q_pools", "k_half_pools", "block_rows",
     "proxy_scores", "sol_route", "route_head", "topk_keep_count", "topk_route",
     "centroid_groups", "centroid_table", "sol_attention_head", "lcsa_mask",
-    "masked_attention_head", "physical_allowed", "resolve_scale",
+    "masked_attention_head", "physical_allowed", "resolve_scale", "virtual_kv_residual_head",
 ]

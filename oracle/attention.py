@@ -30,6 +30,15 @@ Readings:
   mask[b, h mod Hm, i, floor(j/2)]; exact terms only, no centroids; the
   granularity is block-level (no token-causal mask inside a block). A row with
   no allowed block gives o = 0 and lse = -inf.
+* Virtual K/V, residual mode ("Configure H3 Static Virtual KV", the mode
+  list and "What virtual means physically"): queries stay on the physical
+  slices; the physical keys all stay exact; every added virtual slice
+  re-reads one source slice through the logical source map and enters only as
+  skipped-block centroid terms (2x32 on the page) in the same softmax.
+  Reading: a slice is ``slice_tokens`` consecutive tokens, a multiple of 64,
+  so that its blocks are whole source blocks; the source keys are taken as
+  given (INT8 codes and per-block scales of the source), so a temporal phase
+  a caller wants on a virtual slice is already in the source it passes.
 * LCSA mask from frame geometry ("FlashVSR Sparge Attention", intro: each
   query block attends only to a small, locally causal set of key blocks; the
   sampler builds the mask). Reading: a logical 128-token block belongs to the
@@ -116,6 +125,50 @@ def sol_attention_head(q8, q_scale, k8, k_scale, v, keep, centroid_mode: int,
             O[r0:r1] = 0.0
             lse[r0:r1] = -math.inf
             continue
+        O[r0:r1], lse[r0:r1] = _softmax_rows(np.concatenate(logits, axis=1),
+                                             np.concatenate(values, axis=0))
+    return O, lse
+
+
+def virtual_kv_residual_head(q8, q_scale, k8, k_scale, v, src_k8, src_k_scale, src_v,
+                             slice_tokens: int, src_map, centroid_mode: int = 2,
+                             softmax_scale: float = 0.0, q_blocks=None):
+    """Residual virtual K/V attention of one (batch, head).
+
+    Exact terms: every physical key block (k8, k_scale, v). Centroid terms:
+    for each added virtual slice l, the groups of source blocks
+    src_map[l]*bps .. (src_map[l]+1)*bps - 1, bps = slice_tokens / 64, built
+    from (src_k8, src_k_scale, src_v) exactly as a skipped block's are.
+    Returns (O fp64 [Lq, d], lse fp64 [Lq]); rows outside ``q_blocks`` stay NaN.
+    """
+    if slice_tokens <= 0 or slice_tokens % K_ROWS:
+        raise ValueError("slice_tokens must be a positive multiple of 64")
+    n_src = src_k8.shape[0] // slice_tokens
+    if n_src * slice_tokens != src_k8.shape[0]:
+        raise ValueError("the source holds a whole number of slices")
+    if any(not 0 <= s < n_src for s in src_map):
+        raise ValueError("source map entry out of range")
+    Lq, d = q8.shape
+    scale = resolve_scale(d, softmax_scale)
+    v = np.asarray(v, dtype=np.float64)
+    kspans = block_rows(k8.shape[0], K_ROWS)
+    table = centroid_table(src_k8, src_k_scale, src_v, centroid_mode)
+    bps = slice_tokens // K_ROWS
+    virtual = [grp for s in src_map for j in range(s * bps, (s + 1) * bps) for grp in table[j]]
+    O = np.full((Lq, d), np.nan)
+    lse = np.full(Lq, np.nan)
+    qspans = block_rows(Lq, Q_ROWS)
+    for i in (range(len(qspans)) if q_blocks is None else q_blocks):
+        r0, r1 = qspans[i]
+        Qi = q8[r0:r1].astype(np.float64)
+        logits, values = [], []
+        for j, (t0, t1) in enumerate(kspans):
+            dots = Qi @ k8[t0:t1].astype(np.float64).T
+            logits.append((float(q_scale[i]) * float(k_scale[j]) * scale) * dots)
+            values.append(v[t0:t1])
+        for n, kbar, vbar in virtual:
+            logits.append(((float(q_scale[i]) * scale) * (Qi @ kbar) + math.log(n))[:, None])
+            values.append(vbar[None, :])
         O[r0:r1], lse[r0:r1] = _softmax_rows(np.concatenate(logits, axis=1),
                                              np.concatenate(values, axis=0))
     return O, lse

@@ -184,3 +184,98 @@ def test_lcsa_mask_is_causal_and_window_monotone():
     assert m1.diagonal().all()                  # every block sees its own frame
     with pytest.raises(ValueError):
         oracle.lcsa_mask(100, 100, 0, 1)
+
+
+# ---------------------------------------------------------------- virtual K/V, residual mode
+def _virtual_case(name, b=0, h=0):
+    w = workloads.get(name)
+    q, k, v = (t.float().numpy() for t in workloads.head_qkv(w, b, h))
+    ks, vs = (t.float().numpy() for t in workloads.source_kv(w, b, h))
+    r = oracle.route_head(q, k, -math.inf)
+    ks8, kss = oracle.quantize_blocks(ks, 64)
+    return w, r, v, ks8, kss, vs
+
+
+def _materialised(w, r, v, ks8, kss, vs, src_map, mode, replace_by_mean):
+    """Dequantised [physical ; virtual slices] K and V, virtual rows optionally mean-replaced per group."""
+    T = w.slice_tokens
+    Kd = _dequant(r["k8"], r["k_scale"], 64)
+    Ksd = _dequant(ks8, kss, 64)
+    Ks, Vs = [Kd], [np.asarray(v, np.float64)]
+    for s in src_map:
+        kk = Ksd[s * T:(s + 1) * T].copy()
+        vv = np.asarray(vs[s * T:(s + 1) * T], np.float64).copy()
+        if replace_by_mean:
+            g = 64 // mode
+            for g0 in range(0, T, g):
+                kk[g0:g0 + g] = kk[g0:g0 + g].mean(axis=0)
+                vv[g0:g0 + g] = vv[g0:g0 + g].mean(axis=0)
+        Ks.append(kk)
+        Vs.append(vv)
+    return np.concatenate(Ks), np.concatenate(Vs)
+
+
+def test_virtual_residual_without_virtual_slices_is_dense():
+    w, r, v, ks8, kss, vs = _virtual_case("virtual_ragged")
+    O, lse = oracle.virtual_kv_residual_head(r["q8"], r["q_scale"], r["k8"], r["k_scale"], v,
+                                             ks8, kss, vs, w.slice_tokens, (), w.centroid_mode)
+    ref = _sdpa(_dequant(r["q8"], r["q_scale"], 128), _dequant(r["k8"], r["k_scale"], 64), v,
+                1.0 / math.sqrt(w.d))
+    assert np.abs(O - ref).max() <= 1e-12
+
+
+@pytest.mark.parametrize("name,mode", [("virtual_small", 2), ("virtual_small", 1),
+                                       ("virtual_ragged", 2), ("virtual_ragged", 1)])
+def test_virtual_residual_equals_dense_over_mean_replaced_virtual_context(name, mode):
+    # each centroid group of a virtual slice is |g| equal keys at its mean: exactly the ln|g| term
+    w, r, v, ks8, kss, vs = _virtual_case(name, 0, 1)
+    O, lse = oracle.virtual_kv_residual_head(r["q8"], r["q_scale"], r["k8"], r["k_scale"], v,
+                                             ks8, kss, vs, w.slice_tokens, w.virtual_map, mode)
+    K2, V2 = _materialised(w, r, v, ks8, kss, vs, w.virtual_map, mode, True)
+    Qd = _dequant(r["q8"], r["q_scale"], 128)
+    scale = 1.0 / math.sqrt(w.d)
+    assert np.abs(O - _sdpa(Qd, K2, V2, scale)).max() <= 1e-10
+    lg = scale * Qd @ K2.T
+    assert np.abs(lse - torch.logsumexp(torch.from_numpy(lg), dim=1).numpy()).max() <= 1e-10
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_virtual_residual_of_identical_token_groups_is_exact_materialisation(mode):
+    # a source whose groups hold identical tokens: the residual mode equals attention over the
+    # materialised seven-slice context, with no approximation at all
+    w = workloads.get("virtual_ragged")
+    q, k, v = (t.float().numpy() for t in workloads.head_qkv(w, 1, 0))
+    ks, vs = (t.float().numpy().copy() for t in workloads.source_kv(w, 1, 0))
+    g = 64 // mode
+    for g0 in range(0, ks.shape[0], g):
+        ks[g0:g0 + g] = ks[g0]
+        vs[g0:g0 + g] = vs[g0]
+    r = oracle.route_head(q, k, -math.inf)
+    ks8, kss = oracle.quantize_blocks(ks, 64)
+    src_map = (1, 0, 1)
+    O, _ = oracle.virtual_kv_residual_head(r["q8"], r["q_scale"], r["k8"], r["k_scale"], v,
+                                           ks8, kss, vs, w.slice_tokens, src_map, mode)
+    K2, V2 = _materialised(w, r, v, ks8, kss, vs, src_map, mode, False)
+    ref = _sdpa(_dequant(r["q8"], r["q_scale"], 128), K2, V2, 1.0 / math.sqrt(w.d))
+    assert np.abs(O - ref).max() <= 1e-10
+
+
+def test_virtual_residual_map_order_does_not_matter_and_each_slice_counts():
+    w, r, v, ks8, kss, vs = _virtual_case("virtual_small")
+    args = (r["q8"], r["q_scale"], r["k8"], r["k_scale"], v, ks8, kss, vs, w.slice_tokens)
+    O1, l1 = oracle.virtual_kv_residual_head(*args, (0, 1, 1), 2)
+    O2, l2 = oracle.virtual_kv_residual_head(*args, (1, 0, 1), 2)
+    O3, _ = oracle.virtual_kv_residual_head(*args, (0, 1), 2)
+    assert np.abs(O1 - O2).max() <= 1e-12 and np.abs(l1 - l2).max() <= 1e-12
+    assert np.abs(O1 - O3).max() > 1e-4      # a repeated slice adds its terms again
+
+
+def test_virtual_residual_rejects_bad_geometry():
+    w, r, v, ks8, kss, vs = _virtual_case("virtual_small")
+    args = (r["q8"], r["q_scale"], r["k8"], r["k_scale"], v, ks8, kss, vs)
+    with pytest.raises(ValueError):
+        oracle.virtual_kv_residual_head(*args, 100, (0,))
+    with pytest.raises(ValueError):
+        oracle.virtual_kv_residual_head(*args, 320, (2,))
+    with pytest.raises(ValueError):
+        oracle.virtual_kv_residual_head(*args, 256, (0,))

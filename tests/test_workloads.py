@@ -52,3 +52,13 @@ def test_pe_signal_and_prefix():
     kf = k.float().numpy()[256:]
     corr = np.corrcoef(vid.ravel(), kf.ravel())[0, 1]
     assert corr > 0.5
+
+
+def test_virtual_kv_shapes():
+    w = workloads.get("h3_virtual")
+    assert w.Lq == w.Lk == 2 * 48 * 84 == 8064 and w.slice_tokens % 64 == 0
+    assert len(w.virtual_map) == 5 and set(w.virtual_map) <= {0, 1}
+    ks, vs = workloads.source_kv(workloads.get("virtual_ragged"), 0, 1)
+    assert tuple(ks.shape) == (2 * 192, 64) and ks.dtype == torch.bfloat16
+    k_phys = workloads.head_qkv(workloads.get("virtual_small"), 0, 1)[1]
+    assert torch.equal(workloads.source_kv(workloads.get("virtual_small"), 0, 1)[0], k_phys)

@@ -37,11 +37,11 @@ import torch
 
 __all__ = [
     "Workload", "WORKLOADS", "get", "head_qkv", "batch_qkv", "block_mask",
-    "lcsa_block_mask", "pe_table", "W_SEED",
+    "lcsa_block_mask", "pe_table", "W_SEED", "source_kv",
 ]
 
 W_SEED = 7
-_Q, _K, _V = 0, 1, 2
+_Q, _K, _V, _KS, _VS = 0, 1, 2, 3, 4
 
 
 @dataclass(frozen=True)
@@ -62,6 +62,10 @@ class Workload:
     mask: str | None = None          # "lcsa" for the explicit block-mask entry
     frame_tokens: int = 0            # tokens per latent frame (LCSA)
     lcsa_window: int = 2             # key frames allowed: [f_q - window, f_q]
+    slice_tokens: int = 0            # virtual K/V: tokens per latent-time slice
+    virtual_map: tuple = ()          # virtual K/V: source slice of each added virtual slice
+    n_source_slices: int = 0         # virtual K/V: 0 = the physical K/V is the source,
+                                     # else a separate N(0,1) source of this many slices
     seed: int = 0
     notes: str = field(default="", compare=False)
 
@@ -110,6 +114,13 @@ WORKLOADS = {
                    n_prefix=1024, taus=(1.0,), centroid_mode=1, seed=1005,
                    notes="H3-like: 1024 N(0,1) prefix + 21x48x84 video, "
                          "tau=1.0, 1x64"),
+    "h3_virtual": Workload("h3_virtual", 1, 40, 128, _video(2, 48, 84),
+                           _video(2, 48, 84), "pe", grid=(2, 48, 84),
+                           centroid_mode=2, slice_tokens=48 * 84,
+                           virtual_map=(0, 0, 1, 1, 1), seed=1006,
+                           notes="H3 reference-image path: 2 physical latent "
+                                 "slices of 48x84, 5 added virtual slices "
+                                 "re-reading them, 2x32 residuals"),
     # -- small parity cases: several tiles and a ragged tail ----------------
     "ragged_pe": Workload("ragged_pe", 2, 3, 128, 1000, 1000, "pe",
                           grid=(5, 10, 20), taus=(0.5, 1.0), centroid_mode=1,
@@ -130,6 +141,17 @@ WORKLOADS = {
                            5 * 384 + 100, "normal", centroid_mode=0,
                            mask="lcsa", frame_tokens=384, seed=2006,
                            notes="5 frames of 3 logical blocks + ragged tail"),
+    "virtual_small": Workload("virtual_small", 1, 3, 128, _video(2, 10, 32),
+                              _video(2, 10, 32), "pe", grid=(2, 10, 32),
+                              centroid_mode=2, slice_tokens=320,
+                              virtual_map=(0, 1, 1, 0, 1), seed=2007,
+                              notes="2 slices of 320 tokens (5 key blocks)"),
+    "virtual_ragged": Workload("virtual_ragged", 2, 2, 64, 600, 1000, "normal",
+                               centroid_mode=1, slice_tokens=192,
+                               virtual_map=(1, 0, 1, 1), n_source_slices=2,
+                               seed=2008,
+                               notes="ragged queries and keys, separate "
+                                     "2-slice source, 1x64"),
 }
 
 
@@ -188,6 +210,18 @@ def head_qkv(w: Workload, b: int, h: int):
     elif w.gen != "normal":
         raise ValueError(f"unknown generator {w.gen!r}")
     return _bf16(q), _bf16(k), _bf16(v)
+
+
+def source_kv(w: Workload, b: int, h: int):
+    """(k_src, v_src) of one (batch, head) for a virtual K/V workload, bf16 CPU.
+
+    ``n_source_slices == 0``: the physical K and V themselves; otherwise a
+    separate N(0, 1) source of ``n_source_slices * slice_tokens`` tokens."""
+    if w.n_source_slices == 0:
+        _, k, v = head_qkv(w, b, h)
+        return k, v
+    n = w.n_source_slices * w.slice_tokens
+    return _bf16(_normal(w, b, h, _KS, n)), _bf16(_normal(w, b, h, _VS, n))
 
 
 def batch_qkv(w: Workload, heads=None, device="cpu"):
