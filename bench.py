@@ -421,6 +421,72 @@ def lcsa_measure(bsva, steps, warmup, dist, int8_v=False):
             "dense_equiv_tflops": round(w.dense_flops() / (ms * 1e-3) / 1e12, 2)}
 
 
+def virtual_work(w, n_virtual):
+    """Algorithmic FLOPs of one residual virtual K/V call: every physical pair exact, plus one
+    centroid logit and one centroid value row per virtual group and query row."""
+    groups = n_virtual * (w.slice_tokens // 64) * w.centroid_mode
+    pairs = w.B * w.H * w.Lq * (w.Lk + groups)
+    return 2.0 * w.d * pairs, 2.0 * w.d * pairs
+
+
+def virtual_kv_measure(bsva, steps, warmup, dist, peaks):
+    """H3 static virtual K/V, residual mode: quantise the physical Q/K, then the residual entry
+    (dense kept lists, virtual tile table, source centroids, attention)."""
+    w = workloads.get("h3_virtual")
+    Q, K, V = [x.cuda() for x in workloads.batch_qkv(w)]
+    qk = bsva.quantize_qk(Q, K)
+    s = bsva.Shape(w.B, w.H, w.Lq, w.Lk, w.d, 0)
+    n_src = w.Lk // w.slice_tokens
+    ws = torch.zeros(bsva.virtual_kv_workspace_bytes(s, w.slice_tokens, n_src, w.centroid_mode),
+                     dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(Q)
+
+    def one(evs=None):
+        if evs:
+            evs[0].record()
+        bsva.quantize_qk(Q, K, out=qk)
+        if evs:
+            evs[1].record()
+        bsva.virtual_kv_residual_fwd(qk, V, w.slice_tokens, w.virtual_map, centroid_mode=w.centroid_mode,
+                                     workspace=ws, out=out)
+        if evs:
+            evs[2].record()
+
+    for _ in range(warmup):
+        one()
+    _barrier(dist)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    phase = []
+    start.record()
+    for _ in range(steps):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        one(evs)
+        phase.append(evs)
+    end.record()
+    torch.cuda.synchronize()
+    bsva.check_status(ws)
+    ms = _max_over_ranks(dist, start.elapsed_time(end) / steps)
+    q_ms = _max_over_ranks(dist, sum(e[0].elapsed_time(e[1]) for e in phase) / steps)
+    f_ms = _max_over_ranks(dist, sum(e[1].elapsed_time(e[2]) for e in phase) / steps)
+    f_qk, f_pv = virtual_work(w, len(w.virtual_map))
+    p_bf16 = peaks["bf16"] * 1e12
+    t_roof = f_qk / (2.0 * p_bf16) + f_pv / p_bf16
+    peak_eff = (f_qk + f_pv) / t_roof / 1e12
+    achieved = (f_qk + f_pv) / (f_ms * 1e-3) / 1e12
+    n_virtual_tokens = len(w.virtual_map) * w.slice_tokens
+    return {"workload": f"h3_virtual: B=1 H=40 d=128, 2 physical slices of 48x84 (L=8064), "
+                        f"{len(w.virtual_map)} virtual slices re-reading them (map {list(w.virtual_map)}), "
+                        f"2x32 residuals; quantise + residual entry",
+            "ms_per_call": round(ms, 4), "quantize_ms": round(q_ms, 4), "residual_fwd_ms": round(f_ms, 4),
+            "virtual_context_tokens": w.Lk + n_virtual_tokens,
+            "dense_equiv_tflops": round(4.0 * w.d * w.B * w.H * w.Lq * (w.Lk + n_virtual_tokens)
+                                        / (ms * 1e-3) / 1e12, 2),
+            "kept_tflops": round((f_qk + f_pv) / (ms * 1e-3) / 1e12, 2),
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(peak_eff, 2),
+                         "unit": "TFLOP/s", "frac": round(achieved / peak_eff, 4),
+                         "of": "residual entry (centroid build + attention) vs int8 QK + bf16 PV peaks"}}
+
+
 # ------------------------------------------------------------ the oracle --
 def oracle_sample(w, tau, n_route_heads, n_qblocks, seed=0):
     """Time the oracle on a bounded sample; return (extrapolated ms/call, sample text, seconds)."""
@@ -552,6 +618,7 @@ def main():
         del s3
         extra["lcsa_mask_entry"] = lcsa_measure(bsva, max(5, args.steps // 4), 3, dist)
         extra["lcsa_mask_entry_int8_v"] = lcsa_measure(bsva, max(5, args.steps // 4), 3, dist, int8_v=True)
+        extra["virtual_kv_residual"] = virtual_kv_measure(bsva, max(5, args.steps // 4), 3, dist, peaks)
     e2e = None
     if not args.quick:
         Qp, Kp, Vp = Qh.pin_memory(), Kh.pin_memory(), Vh.pin_memory()

@@ -14,6 +14,8 @@ Entry points (same names as the C ABI):
 * ``masked_block_attn_fwd(q8, ..., mask)``   explicit logical 128x128 block mask
 * ``build_lcsa_mask(Lq, Lk, frame_tokens, window)`` that mask from frame geometry, on the device
 * ``quantize_v(v)``, ``masked_block_attn_fwd_v8(...)`` the mask entry on an INT8 V
+* ``virtual_kv_residual_fwd(qk, v, slice_tokens, src_map)`` residual virtual K/V:
+  physical keys exact, each added virtual slice as centroid terms
 """
 from __future__ import annotations
 
@@ -28,10 +30,10 @@ __all__ = [
     "workspace_bytes", "route_workspace_bytes", "quantize_qk", "sparse_attn_route",
     "sparse_attn_route_topk", "build_lcsa_mask", "quantize_v", "masked_block_attn_fwd_v8", "sparse_attn_fwd",
     "masked_block_attn_fwd", "check_status", "selftest_timeout", "new_workspace",
-    "build_centroids", "sparse_attn_core",
+    "build_centroids", "sparse_attn_core", "virtual_kv_workspace_bytes", "virtual_kv_residual_fwd",
 ]
 
-ABI_VERSION = 2
+ABI_VERSION = 3
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
 
@@ -85,6 +87,10 @@ _SIGS = {
                                                 ctypes.c_float, ctypes.c_int, _P, _P, _P, ctypes.c_size_t,
                                                 _P]),
     "bsva_selftest_timeout": (ctypes.c_int, [_P, ctypes.c_size_t, ctypes.c_longlong, _P]),
+    "bsva_virtual_kv_workspace_bytes": (ctypes.c_size_t, [Shape, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "virtual_kv_residual_fwd": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P, _P,
+                                               ctypes.POINTER(ctypes.c_int), ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_float, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
 }
 
 
@@ -410,6 +416,58 @@ def masked_block_attn_fwd_v8(q8, q_scale, k8, k_scale, v8, v_scale, block_mask, 
     _need(v_scale, torch.float32, (B, H, -(-Lk // 64)), "v_scale")
     return _masked_call("masked_block_attn_fwd_v8", q8, q_scale, k8, k_scale, (v8, v_scale), v8, block_mask,
                         softmax_scale, with_lse, workspace, out, lse, out_dtype, stream)
+
+
+def virtual_kv_workspace_bytes(shape: Shape, slice_tokens: int, n_src_slices: int, centroid_mode: int = 2) -> int:
+    n = load().bsva_virtual_kv_workspace_bytes(shape, slice_tokens, n_src_slices, centroid_mode)
+    if n == 0:
+        raise BsvaError(1, f"bad shape or geometry for a virtual K/V workspace: {_fmt(shape)}, "
+                           f"slice_tokens {slice_tokens}, {n_src_slices} source slices, mode {centroid_mode}")
+    return n
+
+
+def virtual_kv_residual_fwd(qk: dict, v: torch.Tensor, slice_tokens: int, src_map, source: dict | None = None,
+                            src_v: torch.Tensor | None = None, centroid_mode: int = 2, softmax_scale: float = 0.0,
+                            with_lse: bool = False, workspace: torch.Tensor | None = None, out=None, lse=None,
+                            out_dtype=torch.bfloat16, stream=None):
+    """Residual virtual K/V attention (C ABI ``virtual_kv_residual_fwd``).
+
+    ``qk`` is the ``quantize_qk`` output of the physical Q and K; ``v`` the
+    physical values. Virtual slice l re-reads slice ``src_map[l]`` of the
+    source: ``source`` (a ``quantize_qk`` output of the source keys, its
+    ``k_scale`` and ``k_pool`` are used) and ``src_v``, by default the
+    physical ``qk`` and ``v`` themselves."""
+    lib = load()
+    B, H, Lq, d = qk["q8"].shape
+    Lk = qk["k8"].shape[2]
+    s = Shape(B, H, Lq, Lk, d, 0)
+    _need(qk["q8"], torch.int8, None, "q8")
+    _need(qk["k8"], torch.int8, (B, H, Lk, d), "k8")
+    _need(v, torch.bfloat16, (B, H, Lk, d), "v")
+    source = qk if source is None else source
+    src_v = v if src_v is None else src_v
+    _need(src_v, torch.bfloat16, None, "src_v")
+    Ls = src_v.shape[2]
+    if slice_tokens <= 0 or Ls % slice_tokens:
+        raise ValueError(f"src_v holds {Ls} tokens, not a whole number of {slice_tokens}-token slices")
+    n_src = Ls // slice_tokens
+    _need(src_v, torch.bfloat16, (B, H, Ls, d), "src_v")
+    _need(source["k_scale"], torch.float32, (B, H, -(-Ls // 64)), "source k_scale")
+    _need(source["k_pool"], torch.int32, (B, H, -(-Ls // 64), 2, d), "source k_pool")
+    src_map = [int(x) for x in src_map]
+    cmap = (ctypes.c_int * len(src_map))(*src_map) if src_map else None
+    if workspace is None:
+        workspace = torch.zeros(virtual_kv_workspace_bytes(s, slice_tokens, n_src, centroid_mode),
+                                dtype=torch.uint8, device=v.device)
+    out = _out(out, (B, H, Lq, d), out_dtype, v.device)
+    if with_lse and lse is None:
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=v.device)
+    _check(lib.virtual_kv_residual_fwd(s, _ptr(qk["q8"]), _ptr(qk["q_scale"]), _ptr(qk["k8"]), _ptr(qk["k_scale"]),
+                                       _ptr(v), slice_tokens, n_src, _ptr(source["k_scale"]), _ptr(source["k_pool"]),
+                                       _ptr(src_v), cmap, len(src_map), centroid_mode, ctypes.c_float(softmax_scale),
+                                       OUT_DTYPES[out.dtype], _ptr(out), _ptr(lse), _ptr(workspace),
+                                       workspace.numel(), _stream(stream)))
+    return (out, lse) if with_lse else out
 
 
 def check_status(workspace: torch.Tensor, stream=None):

@@ -123,7 +123,7 @@ int run_attention(const bsva_shape& s, const int8_t* q8, const float* q_scale, c
                   const float* k_scale, const void* v, const uint8_t* kept_mask, const int32_t* kept_idx,
                   const int32_t* kept_cnt, int centroid_mode, float softmax_scale, int out_dtype, void* out,
                   float* lse, unsigned char* ws, const WsLayout& L, cudaStream_t st,
-                  const float* v_scale = nullptr) {
+                  const float* v_scale = nullptr, const int2* vtab = nullptr) {
   int rc = get_encoder();
   if (rc) return rc;
   const uint64_t BH = uint64_t(s.B) * s.H;
@@ -166,6 +166,8 @@ int run_attention(const bsva_shape& s, const int8_t* q8, const float* q_scale, c
   a.v_scale = v_scale;
   a.cfac = centroid_mode > 0 ? reinterpret_cast<const float*>(ws + L.cfac) : nullptr;
   a.cbias = centroid_mode > 0 ? reinterpret_cast<const float*>(ws + L.cbias) : nullptr;
+  a.vtab = vtab;
+  a.n_vtiles = vtab ? L.n_vtiles : 0;
   a.out = out_dtype == BSVA_OUT_BF16 ? reinterpret_cast<__nv_bfloat16*>(out) : nullptr;
   a.out_f32 = out_dtype == BSVA_OUT_F32 ? reinterpret_cast<float*>(out) : nullptr;
   a.lse = lse;
@@ -437,6 +439,70 @@ int masked_block_attn_fwd_v8(bsva_shape s, const int8_t* q8, const float* q_scal
   if (e != cudaSuccess) return cuda_fail(e, "mask expansion launch");
   return run_attention(s, q8, q_scale, k8, k_scale, v8, nullptr, kidx, kcnt, 0, softmax_scale, out_dtype, out, lse,
                        ws, L, st, v_scale);
+}
+
+static int check_virtual_geometry(int slice_tokens, int n_src_slices, int centroid_mode) {
+  if (slice_tokens < KB || slice_tokens % KB != 0)
+    return fail(BSVA_ERR_INVALID_ARG, "slice_tokens = %d must be a positive multiple of 64", slice_tokens);
+  if (n_src_slices < 1) return fail(BSVA_ERR_INVALID_ARG, "n_src_slices = %d must be >= 1", n_src_slices);
+  if (size_t(slice_tokens) * size_t(n_src_slices) > (size_t(1) << 30))
+    return fail(BSVA_ERR_INVALID_ARG, "source too long: %d slices of %d tokens", n_src_slices, slice_tokens);
+  if (centroid_mode != 1 && centroid_mode != 2)
+    return fail(BSVA_ERR_INVALID_ARG, "centroid_mode = %d; use 1 (1x64) or 2 (2x32)", centroid_mode);
+  return BSVA_OK;
+}
+
+size_t bsva_virtual_kv_workspace_bytes(bsva_shape s, int slice_tokens, int n_src_slices, int centroid_mode) {
+  if (check_shape(s) != BSVA_OK || check_virtual_geometry(slice_tokens, n_src_slices, centroid_mode) != BSVA_OK)
+    return 0;
+  return ws_layout_virtual(s, slice_tokens, n_src_slices, 0, centroid_mode).total;
+}
+
+int virtual_kv_residual_fwd(bsva_shape s, const int8_t* q8, const float* q_scale, const int8_t* k8,
+                            const float* k_scale, const void* v, int slice_tokens, int n_src_slices,
+                            const float* src_k_scale, const int32_t* src_k_pool, const void* src_v,
+                            const int* src_map, int n_virtual, int centroid_mode, float softmax_scale,
+                            int out_dtype, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                            bsva_stream_t stream) {
+  int rc;
+  if ((rc = check_shape(s))) return rc;
+  if ((rc = check_virtual_geometry(slice_tokens, n_src_slices, centroid_mode))) return rc;
+  if (n_virtual < 0 || n_virtual > kMaxVirtualSlices)
+    return fail(BSVA_ERR_INVALID_ARG, "n_virtual = %d outside [0, %d]", n_virtual, kMaxVirtualSlices);
+  if (n_virtual > 0 && src_map == nullptr) return fail(BSVA_ERR_INVALID_ARG, "src_map is NULL");
+  for (int l = 0; l < n_virtual; ++l)
+    if (src_map[l] < 0 || src_map[l] >= n_src_slices)
+      return fail(BSVA_ERR_INVALID_ARG, "src_map[%d] = %d outside [0, %d)", l, src_map[l], n_src_slices);
+  if (std::isnan(softmax_scale) || std::isinf(softmax_scale))
+    return fail(BSVA_ERR_INVALID_ARG, "softmax_scale must be finite");
+  if (out_dtype != BSVA_OUT_BF16 && out_dtype != BSVA_OUT_F32)
+    return fail(BSVA_ERR_INVALID_ARG, "out_dtype = %d; use BSVA_OUT_BF16 (0) or BSVA_OUT_F32 (1)", out_dtype);
+  REQUIRE_PTR(q8, 16); REQUIRE_PTR(q_scale, 4); REQUIRE_PTR(k8, 16); REQUIRE_PTR(k_scale, 4);
+  REQUIRE_PTR(v, 16); REQUIRE_PTR(out, 16);
+  if (n_virtual > 0) {
+    REQUIRE_PTR(src_k_scale, 4); REQUIRE_PTR(src_k_pool, 16); REQUIRE_PTR(src_v, 16);
+  }
+  if (lse && !aligned(lse, 4)) return fail(BSVA_ERR_INVALID_ARG, "lse is not 4-byte aligned");
+  const WsLayout L = ws_layout_virtual(s, slice_tokens, n_src_slices, n_virtual, centroid_mode);
+  if ((rc = check_workspace(workspace, workspace_bytes, L.total))) return rc;
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  int32_t* kidx = reinterpret_cast<int32_t*>(ws + L.kidx);
+  int32_t* kcnt = reinterpret_cast<int32_t*>(ws + L.kcnt);
+  cudaError_t e = launch_dense_lists(s, kidx, kcnt, st);
+  if (e != cudaSuccess) return cuda_fail(e, "dense list launch");
+  if (n_virtual == 0)   // nothing virtual: dense exact attention over the physical keys
+    return run_attention(s, q8, q_scale, k8, k_scale, v, nullptr, kidx, kcnt, 0, softmax_scale, out_dtype, out, lse,
+                         ws, L, st);
+  int2* vtab = reinterpret_cast<int2*>(ws + L.vtab);
+  e = launch_virtual_tiles(src_map, n_virtual, slice_tokens / KB * centroid_mode, vtab, st);
+  if (e != cudaSuccess) return cuda_fail(e, "virtual tile table launch");
+  bsva_shape src = s;
+  src.Lk = slice_tokens * n_src_slices;
+  if ((rc = build_centroids(src, src_k_pool, src_k_scale, src_v, centroid_mode, ws, L, st))) return rc;
+  return run_attention(s, q8, q_scale, k8, k_scale, v, nullptr, kidx, kcnt, centroid_mode, softmax_scale, out_dtype,
+                       out, lse, ws, L, st, nullptr, vtab);
 }
 
 int bsva_check_status(void* workspace, bsva_stream_t stream) {

@@ -35,6 +35,10 @@
 // Centroid tiles hold 32 groups as (hi, lo) INT8 row pairs (pool = 128 hi + lo)
 // so their dot with q8 is exact in int32; the value rows are (bf16 hi, bf16 lo)
 // and share one probability.
+// Virtual K/V, residual mode ("Configure H3 Static Virtual KV", the mode
+// list): the kept lists hold every physical block, and the centroid tiles are
+// those of the added virtual slices, each re-reading its source slice's groups
+// through a per-tile table (a.vtab) instead of a skipped-block mask.
 // Every wait is bounded: on a timeout the CTA records it in the workspace
 // status word, all roles leave their loops, TMEM is freed and the CTA exits.
 #include <cmath>
@@ -94,7 +98,8 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // kV8: V is INT8 with per-block scales (a.v_scale), P and V enter PV as f16.
-template <int D, bool kV8>
+// kVirt: the centroid tiles are the virtual slices' (a.vtab), not the skipped blocks'.
+template <int D, bool kV8, bool kVirt>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_kernel(const AttnArgs a, const __grid_constant__ AttnMaps maps) {
   extern __shared__ unsigned char smem_raw[];
@@ -109,7 +114,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   const size_t row_item = size_t(bh) * a.nQB + i;
 
   const int n_exact = a.kept_cnt[row_item];
-  const int n_cent = (a.centroid_mode > 0 && n_exact < a.nKB) ? a.nCT : 0;
+  // Sol: the whole centroid table once some block is skipped; virtual K/V: the virtual slices' tiles
+  const int n_cent = kVirt ? a.n_vtiles : (a.centroid_mode > 0 && n_exact < a.nKB) ? a.nCT : 0;
   const int N = n_exact + n_cent;
   const int q0 = i * QB;
 
@@ -177,15 +183,26 @@ __global__ void __launch_bounds__(kThreads, 2)
     float chunk_f = 0.f;
     int j_next = 0;              // key block of the K step's tile
     float cf_next = 0.f, cb_next = 0.f;   // centroid metadata of the next centroid tile
+    int cr_next = 0;                      // and its first table row
     bool ok = true;
 
-    // group metadata of centroid tile t for this lane
-    auto cent_meta = [&](int t, float& fac, float& bias) {
-      const int G = t * 32 + lane;
-      const int jb = G / a.centroid_mode;
-      const bool kept = jb >= a.nKB || kmask[jb];
-      fac = sqs * cfac[G];
-      bias = kept ? -INFINITY : cbias[G];
+    // group metadata of centroid tile t for this lane, and the tile's first table row
+    auto cent_meta = [&](int t, float& fac, float& bias, int& row) {
+      if constexpr (kVirt) {   // virtual slice: 32 source groups from e.x, the first e.y of them live
+        const int2 e = a.vtab[t];
+        const bool live = lane < e.y;
+        const int G = e.x + (live ? lane : 0);   // dead lanes re-read a live entry, never past the table
+        fac = sqs * cfac[G];
+        bias = live ? cbias[G] : -INFINITY;
+        row = 2 * e.x;
+      } else {        // Sol: groups 32t .. 32t+31, live where their block was skipped
+        const int G = t * 32 + lane;
+        const int jb = G / a.centroid_mode;
+        const bool kept = jb >= a.nKB || kmask[jb];
+        fac = sqs * cfac[G];
+        bias = kept ? -INFINITY : cbias[G];
+        row = t * KB;
+      }
     };
     auto k_step = [&](int t) -> bool {
       const int sk = t % NK;
@@ -213,14 +230,14 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       } else {
         const int tc = t - n_exact;
-        row = tc * KB;
         float fac, bias;
-        if (tc == 0) cent_meta(0, fac, bias);
-        else { fac = cf_next; bias = cb_next; }
+        if (tc == 0) cent_meta(0, fac, bias, row);
+        else { fac = cf_next; bias = cb_next; row = cr_next; }
+        if constexpr (!kVirt) row = tc * KB;   // Sol: the table in order
         mt.fac[lane] = fac;
         mt.bias[lane] = bias;
         if (lane == 0) mt.centroid = 1;
-        if (t + 1 < N) cent_meta(tc + 1, cf_next, cb_next);   // prefetch the next centroid tile
+        if (t + 1 < N) cent_meta(tc + 1, cf_next, cb_next, cr_next);   // prefetch the next centroid tile
       }
       if (lane == 0) sm.vrow[t % NR] = row;
       __syncwarp();   // the metadata is published by lane 0's arrive on the stage's barrier
@@ -603,21 +620,24 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-template <int D, bool kV8>
+template <int D, bool kV8, bool kVirt>
 cudaError_t launch_attn_dv(const AttnArgs& a, const AttnMaps& maps, cudaStream_t st) {
   // At least 100 KB so that no more than two CTAs share an SM: two 256-column
   // TMEM allocations fill the SM's 512 columns.
   const size_t smem = sizeof(Smem<D>) + 1024 > 100 * 1024 ? sizeof(Smem<D>) + 1024 : 100 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, kV8>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  cudaError_t e =
+      cudaFuncSetAttribute(attn_kernel<D, kV8, kVirt>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   const unsigned grid = unsigned(a.B) * a.H * a.nQB;
-  attn_kernel<D, kV8><<<grid, kThreads, smem, st>>>(a, maps);
+  attn_kernel<D, kV8, kVirt><<<grid, kThreads, smem, st>>>(a, maps);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_attn_d(const AttnArgs& a, const AttnMaps& maps, cudaStream_t st) {
-  return a.v_scale ? launch_attn_dv<D, true>(a, maps, st) : launch_attn_dv<D, false>(a, maps, st);
+  // no entry point combines an INT8 V with virtual slices
+  if (a.vtab) return launch_attn_dv<D, false, true>(a, maps, st);
+  return a.v_scale ? launch_attn_dv<D, true, false>(a, maps, st) : launch_attn_dv<D, false, false>(a, maps, st);
 }
 
 // One CTA waits on a barrier nothing arrives at; the bounded wait runs out.

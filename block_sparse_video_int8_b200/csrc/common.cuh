@@ -27,10 +27,12 @@ struct WsLayout {
   size_t cv = 0;            // bf16  [BH, nCR, d]  centroid values, hi/lo rows
   size_t cfac = 0;          // fp32  [BH, nCG]     sk_j / |g|
   size_t cbias = 0;         // fp32  [BH, nCG]     log2|g| or -inf
-  size_t kidx = 0;          // int32 [BH, nQB, nKB] kept lists (mask entry)
+  size_t kidx = 0;          // int32 [BH, nQB, nKB] kept lists (mask entry, virtual K/V)
   size_t kcnt = 0;          // int32 [BH, nQB]
+  size_t vtab = 0;          // int2  [n_vtiles] virtual K/V: (first source group, live groups) per tile
   size_t total = 0;
   int nCT = 0;              // centroid tiles per head (64 rows = 32 groups each)
+  int n_vtiles = 0;         // virtual K/V: centroid tiles per query block
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -54,6 +56,34 @@ inline WsLayout ws_layout(const bsva_shape& s, int centroid_mode) {
     w.kidx = off;  off = align256(off + BH * nQB * size_t(nKB) * 4);
     w.kcnt = off;  off = align256(off + BH * nQB * 4);
   }
+  w.total = off;
+  return w;
+}
+
+// Virtual K/V (residual mode): the physical keys run as dense kept lists, the
+// centroid table holds the groups of the source slices, and every added
+// virtual slice is ceil(groups per slice / 32) tiles read from its source
+// slice's groups.
+constexpr int kMaxVirtualSlices = 32;
+
+inline WsLayout ws_layout_virtual(const bsva_shape& s, int slice_tokens, int n_src, int n_virtual,
+                                  int centroid_mode) {
+  WsLayout w;
+  const size_t BH = size_t(s.B) * s.H;
+  const int nQB = (s.Lq + QB - 1) / QB, nKB = (s.Lk + KB - 1) / KB;
+  const int gps = slice_tokens / KB * centroid_mode;     // groups per slice
+  const int tps = (gps + 31) / 32;                       // tiles per virtual slice
+  w.nCT = (n_src * gps + 31) / 32;
+  w.n_vtiles = n_virtual * tps;
+  const size_t nCR = size_t(w.nCT) * 64, nCG = size_t(w.nCT) * 32;
+  size_t off = 256;
+  w.kidx = off;  off = align256(off + BH * nQB * size_t(nKB) * 4);
+  w.kcnt = off;  off = align256(off + BH * nQB * 4);
+  w.vtab = off;  off = align256(off + size_t(kMaxVirtualSlices) * tps * 8);
+  w.ck8 = off;   off = align256(off + BH * nCR * s.d);
+  w.cv = off;    off = align256(off + BH * nCR * s.d * 2);
+  w.cfac = off;  off = align256(off + BH * nCG * 4);
+  w.cbias = off; off = align256(off + BH * nCG * 4);
   w.total = off;
   return w;
 }
@@ -303,6 +333,8 @@ struct AttnArgs {
   const float* v_scale;     // [BH, nKB] per-block scales of an INT8 V (mask entry), null for bf16 V
   const float* cfac;        // [BH, nCT*32]
   const float* cbias;       // [BH, nCT*32]
+  const int2* vtab;         // virtual K/V: [n_vtiles] (first source group, live groups); null otherwise
+  int n_vtiles;             // virtual K/V: centroid tiles of every query block
   __nv_bfloat16* out;       // [BH, Lq, d] bf16 output, or
   float* out_f32;           // [BH, Lq, d] fp32 output (exactly one is non-null)
   float* lse;               // [BH, Lq] nullable
@@ -332,6 +364,11 @@ cudaError_t launch_lcsa_mask(int Lq, int Lk, int frame_tokens, int window, int b
                              cudaStream_t st);
 cudaError_t launch_mask_expand(const bsva_shape& s, const uint8_t* block_mask, int mask_heads, int32_t* kept_idx,
                                int32_t* kept_cnt, cudaStream_t st);
+// Kept lists with every key block of every query block (virtual K/V: the physical keys stay exact).
+cudaError_t launch_dense_lists(const bsva_shape& s, int32_t* kept_idx, int32_t* kept_cnt, cudaStream_t st);
+// The virtual-tile table from a source map of n_virtual <= kMaxVirtualSlices host entries.
+cudaError_t launch_virtual_tiles(const int* src_map, int n_virtual, int groups_per_slice, int2* vtab,
+                                 cudaStream_t st);
 cudaError_t launch_attention(const AttnArgs& a, const AttnMaps& maps, cudaStream_t st);
 cudaError_t launch_selftest_timeout(uint32_t* status, uint64_t limit_ns, cudaStream_t st);
 

@@ -1,4 +1,5 @@
-// mask_expand.cu -- logical 128x128 block mask -> physical kept-block lists.
+// mask_expand.cu -- logical 128x128 block mask -> physical kept-block lists,
+// and the kept lists and centroid-tile table of the virtual K/V mode.
 //
 // Method ("FlashVSR Sparge Attention", How it works): routing happens on
 // logical 128-query x 128-key blocks and the mask is converted to the
@@ -14,6 +15,13 @@
 // small, locally causal set of key blocks): a 128-token block belongs to the
 // frame of its first token, floor(128 x / frame_tokens), and key block x_k is
 // allowed for query block x_q iff f_q - window <= f_k <= f_q.
+//
+// Virtual K/V, residual mode ("Configure H3 Static Virtual KV", the mode
+// list): the two real slices stay dense, so dense_lists_kernel writes kept
+// lists holding every key block; virtual_tiles_kernel turns the logical
+// source map (virtual slice l re-reads source slice src[l]) into one entry per
+// centroid tile: the tile's first source group and how many of its 32 groups
+// belong to the slice.
 #include <algorithm>
 
 #include "common.cuh"
@@ -53,7 +61,48 @@ __global__ void __launch_bounds__(256) lcsa_mask_kernel(uint8_t* __restrict__ ma
   }
 }
 
+__global__ void __launch_bounds__(256) dense_lists_kernel(int32_t* __restrict__ kidx, int32_t* __restrict__ kcnt,
+                                                          int nKB, size_t total) {
+  for (size_t idx = size_t(blockIdx.x) * blockDim.x + threadIdx.x; idx < total; idx += size_t(gridDim.x) * blockDim.x) {
+    const int j = int(idx % nKB);
+    kidx[idx] = j;
+    if (j == 0) kcnt[idx / nKB] = nKB;
+  }
+}
+
+// The map travels by value; it is read with compile-time indices only.
+struct VirtualMap {
+  int src[kMaxVirtualSlices];
+};
+
+__global__ void __launch_bounds__(128) virtual_tiles_kernel(VirtualMap m, int n_virtual, int gps, int2* __restrict__ vtab) {
+  const int tps = (gps + 31) / 32;
+#pragma unroll
+  for (int l = 0; l < kMaxVirtualSlices; ++l) {
+    if (l < n_virtual) {
+      for (int lt = threadIdx.x; lt < tps; lt += blockDim.x)
+        vtab[l * tps + lt] = make_int2(m.src[l] * gps + 32 * lt, min(32, gps - 32 * lt));
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_dense_lists(const bsva_shape& s, int32_t* kept_idx, int32_t* kept_cnt, cudaStream_t st) {
+  const int nQB = (s.Lq + QB - 1) / QB, nKB = (s.Lk + KB - 1) / KB;
+  const size_t total = size_t(s.B) * s.H * nQB * nKB;
+  const unsigned grid = unsigned(std::min<size_t>((total + 255) / 256, 148 * 16));
+  dense_lists_kernel<<<grid, 256, 0, st>>>(kept_idx, kept_cnt, nKB, total);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_virtual_tiles(const int* src_map, int n_virtual, int groups_per_slice, int2* vtab,
+                                 cudaStream_t st) {
+  VirtualMap m{};
+  for (int l = 0; l < n_virtual && l < kMaxVirtualSlices; ++l) m.src[l] = src_map[l];
+  virtual_tiles_kernel<<<1, 128, 0, st>>>(m, n_virtual, groups_per_slice, vtab);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_lcsa_mask(int Lq, int Lk, int frame_tokens, int window, int batch, uint8_t* mask,
                              cudaStream_t st) {

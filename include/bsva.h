@@ -10,7 +10,9 @@
  * A second entry point runs an explicit logical 128x128 block mask such as
  * FlashVSR's LCSA streaming mask, with no centroids ("FlashVSR Sparge
  * Attention", intro and How it works; "FlashVSR Kitchen Sparse Attention",
- * intro).
+ * intro). A third runs the residual mode of a static virtual K/V context:
+ * the physical keys exact, every added virtual slice as centroid terms
+ * ("Configure H3 Static Virtual KV", the mode list).
  *
  * Conventions shared by every entry point
  *  - Tensors are contiguous row-major: Q, O [B, H, Lq, d]; K, V [B, H, Lk, d].
@@ -37,7 +39,7 @@
 extern "C" {
 #endif
 
-#define BSVA_ABI_VERSION 2
+#define BSVA_ABI_VERSION 3
 
 enum bsva_status {
   BSVA_OK = 0,
@@ -254,6 +256,50 @@ int masked_block_attn_fwd_v8(bsva_shape s, const int8_t* q8, const float* q_scal
                              float softmax_scale, int out_dtype, void* out,
                              float* lse, void* workspace, size_t workspace_bytes,
                              bsva_stream_t stream);
+
+/* Workspace bytes for virtual_kv_residual_fwd (0 on a bad shape or
+ * geometry); independent of the source map and of n_virtual. */
+size_t bsva_virtual_kv_workspace_bytes(bsva_shape s, int slice_tokens,
+                                       int n_src_slices, int centroid_mode);
+
+/* Residual mode of a static virtual K/V context ("Configure H3 Static Virtual
+ * KV", the mode list and "What virtual means physically"): queries and
+ * outputs stay on the physical rows; every physical key block is an exact
+ * term (the real slices stay dense); each added virtual slice l re-reads
+ * source slice src_map[l] through the logical source map and enters the same
+ * online softmax only as skipped-block centroid terms (2x32 on the page: two
+ * 32-token centroids per 64-token block, log-count |g| in the logit). Nothing
+ * of the virtual context is materialised: the centroid table is built once
+ * per source slice and every virtual tile reads it through the map.
+ *   q8, q_scale, k8, k_scale  physical Q/K as written by bsva_quantize_qk
+ *   v              bf16 [B,H,Lk,d], the physical values
+ *   slice_tokens   tokens per latent-time slice, a positive multiple of 64,
+ *                  so a slice is a whole number of key blocks
+ *   n_src_slices   slices in the source, which holds n_src_slices *
+ *                  slice_tokens tokens per head
+ *   src_k_scale, src_k_pool  fp32 [B,H,nSB], int32 [B,H,nSB,2,d] of the
+ *                  source keys as written by bsva_quantize_qk (nSB =
+ *                  n_src_slices * slice_tokens / 64). With Lk = n_src_slices *
+ *                  slice_tokens the physical k_scale and k_pool serve.
+ *   src_v          bf16 [B,H,n_src_slices*slice_tokens,d] source values (v
+ *                  itself in that case). The keys are used as given: a
+ *                  temporal phase wanted on a virtual slice must already be
+ *                  in the source passed here.
+ *   src_map        HOST array of n_virtual entries in [0, n_src_slices);
+ *                  read during the call only. n_virtual in [0, 32]; 0 gives
+ *                  dense exact attention over the physical keys.
+ *   centroid_mode  2 (2x32) or 1 (1x64)
+ *   workspace      >= bsva_virtual_kv_workspace_bytes(...) bytes, 256-aligned.
+ *   Other arguments as in sparse_attn_fwd. BSVA_ERR_INVALID_ARG for a bad
+ *   geometry, map entry or pointer; nothing is launched then.               */
+int virtual_kv_residual_fwd(bsva_shape s, const int8_t* q8, const float* q_scale,
+                            const int8_t* k8, const float* k_scale,
+                            const void* v, int slice_tokens, int n_src_slices,
+                            const float* src_k_scale, const int32_t* src_k_pool,
+                            const void* src_v, const int* src_map, int n_virtual,
+                            int centroid_mode, float softmax_scale, int out_dtype,
+                            void* out, float* lse, void* workspace,
+                            size_t workspace_bytes, bsva_stream_t stream);
 
 /* masked_block_attn_fwd without a workspace. The source pages have no
  * counterpart: this entry point is for callers that cannot allocate device

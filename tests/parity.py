@@ -237,3 +237,57 @@ def masked_parity_v8(bsva, w, mask, heads=None, q_blocks=None, softmax_scale=0.0
                                                       allowed, softmax_scale, q_blocks=blocks)
         compare_rows(to_np(out[b, h].float()), to_np(lse[b, h]), O_ref, lse_ref, q_rows(w.Lq, blocks), rep)
     return out, lse, rep
+
+
+def source_batch(w, device="cuda"):
+    """[B, H, Ls, d] bf16 source K and V of a virtual K/V workload with a separate source."""
+    n = w.n_source_slices * w.slice_tokens
+    KS = torch.zeros((w.B, w.H, n, w.d), dtype=torch.bfloat16)
+    VS = torch.zeros((w.B, w.H, n, w.d), dtype=torch.bfloat16)
+    for b in range(w.B):
+        for h in range(w.H):
+            ks, vs = workloads.source_kv(w, b, h)
+            KS[b, h].copy_(ks)
+            VS[b, h].copy_(vs)
+    return KS.to(device), VS.to(device)
+
+
+def virtual_parity(bsva, w, heads=None, q_blocks=None, centroid_mode=None, src_map=None, softmax_scale=0.0):
+    """Residual virtual K/V: the GPU quantises the physical Q/K (and a separate source's keys, through
+    the K half of quantize_qk) and runs the entry; the oracle quantises with its own quantiser (checked
+    bit for bit) and computes each head from the same bf16 inputs."""
+    mode = w.centroid_mode if centroid_mode is None else centroid_mode
+    src_map = tuple(w.virtual_map if src_map is None else src_map)
+    Q, K, V = inputs(w)
+    qk = bsva.quantize_qk(Q, K)
+    source = src_v = None
+    if w.n_source_slices:
+        KS, src_v = source_batch(w)
+        source = bsva.quantize_qk(KS, KS)
+    out, lse = bsva.virtual_kv_residual_fwd(qk, V, w.slice_tokens, src_map, source=source, src_v=src_v,
+                                            centroid_mode=mode, softmax_scale=softmax_scale, with_lse=True,
+                                            out_dtype=torch.float32)
+    out16 = bsva.virtual_kv_residual_fwd(qk, V, w.slice_tokens, src_map, source=source, src_v=src_v,
+                                         centroid_mode=mode, softmax_scale=softmax_scale)
+    torch.cuda.synchronize()
+    assert torch.equal(out16, out.to(torch.bfloat16)), "bf16 output != round(fp32 output)"
+    heads = heads or [(b, h) for b in range(w.B) for h in range(w.H)]
+    rep = Report()
+    for b, h in heads:
+        q, k, v = head_np(w, b, h)
+        ref = oracle.route_head(q, k, -math.inf, 0)
+        assert np.array_equal(to_np(qk["q8"][b, h]), ref["q8"]), "q8 differs"
+        assert np.array_equal(to_np(qk["k8"][b, h]), ref["k8"]), "k8 differs"
+        if source is None:
+            ks8, kss, vs = ref["k8"], ref["k_scale"], v
+        else:
+            ks, vs = (t.float().numpy() for t in workloads.source_kv(w, b, h))
+            ks8, kss = oracle.quantize_blocks(ks, 64)
+            assert np.array_equal(to_np(source["k8"][b, h]), ks8), "source k8 differs"
+            assert np.array_equal(to_np(source["k_scale"][b, h]), kss), "source k_scale differs"
+        blocks = list(range(w.nQB)) if q_blocks is None else [i for i in q_blocks if i < w.nQB]
+        O_ref, lse_ref = oracle.virtual_kv_residual_head(ref["q8"], ref["q_scale"], ref["k8"], ref["k_scale"], v,
+                                                         ks8, kss, vs, w.slice_tokens, src_map, mode,
+                                                         softmax_scale, q_blocks=blocks)
+        compare_rows(to_np(out[b, h].float()), to_np(lse[b, h]), O_ref, lse_ref, q_rows(w.Lq, blocks), rep)
+    return out, lse, rep

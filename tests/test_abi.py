@@ -32,7 +32,7 @@ def test_library_builds_and_exports_every_declared_symbol():
 
 
 def test_abi_version_matches_binding():
-    assert bsva.abi_version() == bsva.ABI_VERSION == 2
+    assert bsva.abi_version() == bsva.ABI_VERSION == 3
 
 
 def test_workspace_size_arithmetic():
@@ -137,6 +137,39 @@ def test_fwd_rejects_bad_mode_and_small_workspace():
     assert rc == 1                                                 # mask_heads not in {1, H}
 
 
+def _raw_virtual(s, slice_tokens, n_src, src_map, mode=2, ws_bytes=1 << 30, ptr=0x10000):
+    lib = bsva.load()
+    P = ctypes.c_void_p(ptr)
+    cmap = (ctypes.c_int * len(src_map))(*src_map) if src_map else None
+    return lib.virtual_kv_residual_fwd(s, P, P, P, P, P, slice_tokens, n_src, P, P, P, cmap, len(src_map), mode,
+                                       ctypes.c_float(0), 0, P, None, P, ws_bytes, None)
+
+
+def test_virtual_kv_entry_rejects_bad_geometry_and_workspace():
+    lib = bsva.load()
+    s = bsva.Shape(1, 40, 8064, 8064, 128, 0)
+    # workspace: kept lists of every physical block, the virtual tile table and a
+    # centroid table over the source groups only
+    n = bsva.virtual_kv_workspace_bytes(s, 4032, 2, 2)
+    nQB, nKB, BH = 63, 126, 40
+    nCT = math.ceil(2 * 63 * 2 / 32)
+    assert n >= BH * nQB * nKB * 4 + BH * nCT * 64 * 128 * 3 + BH * nCT * 32 * 8
+    assert n < BH * nQB * nKB * 4 + BH * (nCT + 1) * 64 * 128 * 3 + BH * (nCT + 1) * 32 * 8 + 64 * 1024
+    for bad in ((100, 2, 2), (0, 2, 2), (4032, 0, 2), (4032, 2, 3)):
+        assert lib.bsva_virtual_kv_workspace_bytes(s, *bad) == 0
+    assert _raw_virtual(s, 4000, 2, (0, 1)) == 1 and b"slice_tokens" in lib.bsva_last_error()
+    assert _raw_virtual(s, 4032, 2, (0, 2)) == 1 and b"src_map[1]" in lib.bsva_last_error()
+    assert _raw_virtual(s, 4032, 2, (0, -1)) == 1
+    assert _raw_virtual(s, 4032, 2, tuple([0] * 33)) == 1           # more than 32 virtual slices
+    assert _raw_virtual(s, 4032, 2, (0, 1), mode=3) == 1
+    assert _raw_virtual(s, 4032, 2, (0, 1), ptr=0x10001) == 1       # misaligned
+    assert _raw_virtual(s, 4032, 2, (0, 1), ws_bytes=256) == 3
+    P = ctypes.c_void_p(0x10000)
+    rc = lib.virtual_kv_residual_fwd(s, P, P, P, P, P, 4032, 2, None, P, P, None, 2, 2,
+                                     ctypes.c_float(0), 0, P, None, P, 1 << 30, None)
+    assert rc == 1                                                  # NULL map with n_virtual > 0
+
+
 def test_no_device_is_an_error_not_a_fallback():
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
@@ -146,6 +179,7 @@ def test_no_device_is_an_error_not_a_fallback():
     rc = lib.bsva_quantize_qk(s, P, P, P, P, P, P, P, P, None)
     assert rc in (2, 4)
     assert lib.bsva_last_error()
+    assert _raw_virtual(bsva.Shape(1, 2, 640, 640, 128, 0), 320, 2, (0, 1, 1)) in (2, 4)
 
 
 def test_binding_refuses_cpu_tensors():

@@ -54,3 +54,12 @@ def test_roofline_numbers_are_consistent():
     assert abs(rf["attn"]["frac"] - 1.5) < 1e-4
     assert abs(rf["kept_tflops"] - 2e12 / 1.25e-3 / 1e12) < 0.01
     assert abs(rf["route"]["achieved"] - bench.route_bytes(w) / 1e-4 / 1e9) < 0.1
+
+
+def test_virtual_work_counts_exact_pairs_and_virtual_groups():
+    w = workloads.get("h3_virtual")
+    f_qk, f_pv = bench.virtual_work(w, 5)
+    # 8064 x 8064 exact pairs per head, plus 5 slices x 63 blocks x 2 groups centroid terms per row
+    per_head = 8064 * (8064 + 5 * 63 * 2)
+    assert f_qk == f_pv == 2 * 128 * 40 * per_head
+    assert bench.virtual_work(w, 0)[0] == 2 * 128 * 40 * 8064 * 8064

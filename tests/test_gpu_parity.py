@@ -14,7 +14,7 @@ import torch
 import oracle
 import workloads
 from parity import (Report, assert_within, compare_rows, head_np, inputs, masked_parity, masked_parity_v8,
-                    q_rows, sol_parity, to_np, topk_parity)
+                    q_rows, sol_parity, to_np, topk_parity, virtual_parity)
 
 pytestmark = pytest.mark.gpu
 
@@ -166,6 +166,23 @@ def test_binding_rejects_bad_inputs(gpu_lib):
         gpu_lib.sparse_attn_route(q, q, 1.0, n_prefix=100)
 
 
+@pytest.mark.parametrize("name,mode", [("virtual_small", 2), ("virtual_small", 1), ("virtual_ragged", 2),
+                                       ("virtual_ragged", 1)])
+def test_virtual_kv_small_full_compare(gpu_lib, name, mode):
+    w = workloads.get(name)
+    _, _, rep = virtual_parity(gpu_lib, w, centroid_mode=mode)
+    print(f"{name} mode={mode}: {rep}")
+    assert_within(rep, f"{name} virtual K/V mode {mode}")
+
+
+@pytest.mark.parametrize("src_map", [(), (1,), (0, 1) * 16])
+def test_virtual_kv_map_edges(gpu_lib, src_map):
+    # no virtual slice (dense exact attention), one slice, and the maximum of 32
+    w = workloads.get("virtual_small")
+    _, _, rep = virtual_parity(gpu_lib, w, src_map=src_map, softmax_scale=0.1)
+    assert_within(rep, f"virtual K/V map {src_map}")
+
+
 # ---------------------------------------------------------------- full size
 def _sample_blocks(nQB, n_extra=4, seed=0):
     rng = np.random.default_rng(seed)
@@ -181,6 +198,15 @@ def test_full_lcsa_v8(gpu_lib):
     _, _, rep = masked_parity_v8(gpu_lib, w, workloads.block_mask(w), heads=heads,
                                  q_blocks=_sample_blocks(w.nQB))
     assert_within(rep, "lcsa full INT8 V")
+
+
+@pytest.mark.slow
+def test_full_virtual_kv(gpu_lib):
+    w = workloads.get("h3_virtual")
+    heads = [(0, 0), (0, w.H - 1)]
+    _, _, rep = virtual_parity(gpu_lib, w, heads=heads, q_blocks=_sample_blocks(w.nQB))
+    print(f"h3_virtual: {rep}")
+    assert_within(rep, "h3 virtual K/V residual")
 
 
 @pytest.mark.slow
