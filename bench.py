@@ -298,6 +298,31 @@ def measured_traffic(workload: str):
     return val if (src == attn_source_hash() and val is not None) else None
 
 
+MUFU_EX2_PER_SM_CLK = 16       # ex2.approx per SM per clock (measured with an investigation kernel)
+B200_SMS = 148
+B200_MAX_SM_MHZ = 1965.0
+HBM_SPEC_GBS = 8000.0          # nominal HBM3e figure, beside the measured copy bandwidth
+
+
+def centroid_bytes(w):
+    """Algorithmic HBM bytes of the centroid phase: read V once, write the table
+    (INT8 hi/lo key rows, bf16 hi/lo value rows, factor and log-count per group)."""
+    BH = w.B * w.H
+    groups = w.nKB * w.centroid_mode
+    n_ct = -(-groups // 32)
+    return 2 * BH * w.Lk * w.d + BH * n_ct * 64 * w.d * 3 + BH * n_ct * 32 * 8
+
+
+def mufu_bound(work, w, t_ms):
+    """Secondary ceiling of the attention kernel: one exponential per logit (every kept pair and
+    every centroid term) at the MUFU rate, 16 per SM per clock at the maximum SM clock."""
+    exps = work["f_qk"] / (2.0 * w.d)
+    rate = MUFU_EX2_PER_SM_CLK * B200_SMS * B200_MAX_SM_MHZ * 1e6
+    t_bound = exps / rate
+    return dict(bound="mufu", exps=exps, peak_per_s=rate, t_bound_ms=round(t_bound * 1e3, 4),
+                frac=round(t_bound / (t_ms * 1e-3), 4))
+
+
 def roofline_numbers(w, work, r, peaks):
     p_bf16 = peaks["bf16"] * 1e12
     p_int8 = 2.0 * p_bf16                       # nominal dense INT8 : bf16 ratio on B200
@@ -312,7 +337,12 @@ def roofline_numbers(w, work, r, peaks):
                   frac=round(achieved / peak_eff, 4), traffic=measured_traffic(w.name)),
         route=dict(bound="hbm", achieved=round(rb / (r["route_ms"] * 1e-3) / 1e9, 1), peak=peaks["hbm"],
                    unit="GB/s", frac=round(rb / (r["route_ms"] * 1e-3) / 1e9 / peaks["hbm"], 4),
-                   bytes=rb),
+                   bytes=rb, frac_of_spec=round(rb / (r["route_ms"] * 1e-3) / 1e9 / HBM_SPEC_GBS, 4)),
+        centroids=dict(bound="hbm", achieved=round(centroid_bytes(w) / (r["centroid_ms"] * 1e-3) / 1e9, 1),
+                       peak=peaks["hbm"], unit="GB/s",
+                       frac=round(centroid_bytes(w) / (r["centroid_ms"] * 1e-3) / 1e9 / peaks["hbm"], 4),
+                       bytes=centroid_bytes(w)),
+        mufu=mufu_bound(work, w, r["attn_ms"]),
         dense_equiv_tflops=round(w.dense_flops() / (r["ms"] * 1e-3) / 1e12, 2),
         kept_tflops=round(flops / (r["ms"] * 1e-3) / 1e12, 2),
     )
@@ -484,7 +514,8 @@ def virtual_kv_measure(bsva, steps, warmup, dist, peaks):
             "kept_tflops": round((f_qk + f_pv) / (ms * 1e-3) / 1e12, 2),
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(peak_eff, 2),
                          "unit": "TFLOP/s", "frac": round(achieved / peak_eff, 4),
-                         "of": "residual entry (centroid build + attention) vs int8 QK + bf16 PV peaks"}}
+                         "of": "residual entry (centroid build + attention) vs int8 QK + bf16 PV peaks"},
+            "mufu_bound": mufu_bound(dict(f_qk=f_qk), w, f_ms)}
 
 
 # ------------------------------------------------------------ the oracle --
@@ -645,6 +676,8 @@ def main():
         "kept_tflops": roof["kept_tflops"] * world,
         "roofline": roof["attn"],
         "route_roofline": roof["route"],
+        "centroid_roofline": roof["centroids"],
+        "attn_mufu_bound": roof["mufu"],
         "peaks": {"bf16_tflops": peaks["bf16"], "int8_tops": 2 * peaks["bf16"], "hbm_gbs": peaks["hbm"],
                   "source": f"{peaks['src']} (MEASURED_PEAKS.json burst bf16; int8 = 2x, nominal ratio)"},
         "tau_sweep": sweep,

@@ -46,7 +46,7 @@ def test_route_bytes_formula_at_the_headline_shape():
 def test_roofline_numbers_are_consistent():
     w = workloads.get("tiny")
     work = dict(f_qk=1e12, f_pv=1e12)
-    r = dict(attn_ms=1.0, route_ms=0.1, ms=1.25)
+    r = dict(attn_ms=1.0, route_ms=0.1, centroid_ms=0.05, ms=1.25)
     rf = bench.roofline_numbers(w, work, r, dict(bf16=1000.0, hbm=6000.0, src="test"))
     # int8 at twice the bf16 peak on one tensor pipe: t_roof = 1e12/2e15 + 1e12/1e15 = 1.5 ms
     assert abs(rf["attn"]["peak"] - 2e12 / 1.5e-3 / 1e12) < 0.01
@@ -54,6 +54,19 @@ def test_roofline_numbers_are_consistent():
     assert abs(rf["attn"]["frac"] - 1.5) < 1e-4
     assert abs(rf["kept_tflops"] - 2e12 / 1.25e-3 / 1e12) < 0.01
     assert abs(rf["route"]["achieved"] - bench.route_bytes(w) / 1e-4 / 1e9) < 0.1
+    assert abs(rf["route"]["frac_of_spec"] * 8000.0 - rf["route"]["achieved"]) < 0.5
+
+
+def test_centroid_bytes_and_mufu_bound_at_the_headline_shape():
+    w = workloads.get("wan14b")
+    # V read once (40 x 32760 x 128 bf16) + 32 tiles of 64 rows x (int8 key + bf16 value) + 8 B per group
+    assert bench.centroid_bytes(w) == 2 * 40 * 32760 * 128 + 40 * 32 * 64 * 128 * 3 + 40 * 32 * 32 * 8
+    # one exponential per logit: f_qk / (2 d); 16 per SM per clock on 148 SMs at 1965 MHz
+    work = dict(f_qk=2.0 * 128 * 1e9, f_pv=0.0)
+    mb = bench.mufu_bound(work, w, 2.0)
+    assert mb["exps"] == 1e9
+    assert abs(mb["t_bound_ms"] - 1e9 / (16 * 148 * 1965e6) * 1e3) < 1e-4
+    assert abs(mb["frac"] - mb["t_bound_ms"] / 2.0) < 1e-3
 
 
 def test_virtual_work_counts_exact_pairs_and_virtual_groups():
