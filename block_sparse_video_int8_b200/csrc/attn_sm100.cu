@@ -462,10 +462,11 @@ __global__ void __launch_bounds__(kThreads, 2)
           for (int c = 0; c < 64; ++c)
             if (c >= nvalid) xs[c] = -INFINITY;
         }
-        // P = 2^(x*f - m) as bf16 pairs; lsum adds the bf16-rounded weights
-        // the PV product uses, esum the unrounded ones (log-sum-exp only).
-        // INT8 V: the weights carry the V block scale, P' = 2^(y + log2 s_j), and the sums
-        // take P' * 2^-(log2 s_j), so both sides of O / l see the same (rounded) weights.
+        // P = 2^(x*f - m) as bf16 pairs; lsum adds the fp32 weights before rounding (the
+        // bf16 rounding of each weight, at most 2^-9 relative and unbiased, stays in the
+        // numerator only), and the log-sum-exp uses the same sum.
+        // INT8 V: the weights carry the V block scale, P' = 2^(y + log2 s_j), and lsum takes the
+        // f16-rounded P' * 2^-(log2 s_j) (esum the unrounded weights, log-sum-exp only).
         const float vlog2 = kV8 ? mt.vlog2 : 0.f;
         const float vinv = kV8 ? ex2(-vlog2) : 1.f;
         auto exps = [&](float m_use) {
@@ -481,14 +482,14 @@ __global__ void __launch_bounds__(kThreads, 2)
               pk[c] = pack_f16x2(p0, p1);
               const __half2 h = *reinterpret_cast<const __half2*>(&pk[c]);
               la = __fadd2_rn(la, __half22float2(h));
+              if (want_lse) ea = __fadd2_rn(ea, make_float2(p0, p1));
             } else {
               pk[c] = pack_bf16x2(p0, p1);
-              la = __fadd2_rn(la, make_float2(__uint_as_float(pk[c] << 16), __uint_as_float(pk[c] & 0xFFFF0000u)));
+              la = __fadd2_rn(la, make_float2(p0, p1));
             }
-            if (want_lse) ea = __fadd2_rn(ea, make_float2(p0, p1));
           }
           lsum = la.x + la.y;
-          esum = ea.x + ea.y;
+          esum = kV8 ? ea.x + ea.y : lsum;
           if constexpr (kV8) {
             lsum *= vinv;
             esum *= vinv;
@@ -564,9 +565,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int g = 0; g < 32; ++g) {
           const float p = ex2(xs[g] - m_use);
           pk[g] = pack_bf16x2(p, p);
-          lsum += __uint_as_float(pk[g] << 16);
-          if (want_lse) esum += p;
+          lsum += p;
         }
+        esum = lsum;
       }
       l += lsum;
       le += esum;
