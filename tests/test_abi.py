@@ -186,3 +186,17 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros((1, 1, 128, 64), dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         bsva.sparse_attn_route(q, q, 1.0)
+
+
+def test_binding_signatures_cover_exactly_the_declared_entry_points():
+    # every ctypes signature names a declared symbol, and every declared symbol has a signature
+    assert set(bsva._SIGS) == set(_declared())
+
+
+def test_virtual_kv_binding_refuses_cpu_tensors():
+    q8 = torch.zeros((1, 1, 640, 128), dtype=torch.int8)
+    qk = dict(q8=q8, q_scale=torch.zeros((1, 1, 5)), k8=q8.clone(), k_scale=torch.zeros((1, 1, 10)),
+              k_pool=torch.zeros((1, 1, 10, 2, 128), dtype=torch.int32))
+    v = torch.zeros((1, 1, 640, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        bsva.virtual_kv_residual_fwd(qk, v, 320, (0, 1))
