@@ -72,6 +72,26 @@ def test_prefix_protection():
     assert np.allclose(stats[2:, :2], sub_stats[2:, :2], rtol=0, atol=0)
 
 
+def test_near_threshold_band_is_relative_to_sigma():
+    # mean 0 exactly (symmetric pairs), sigma ~ 577, tau = 0 -> T = 0; the band is 1e-6 sigma ~ 5.8e-4 wide
+    s = np.array([[-1000.0, 1000.0, 1e-4, -1e-4, 1e-2, -1e-2]])
+    keep, stats, band = oracle.sol_route(s, 0.0)
+    assert stats[0, 0] == 0.0 and stats[0, 2] == 0.0
+    assert abs(stats[0, 1] - statistics.pstdev(s[0].tolist())) <= 1e-9
+    assert band[0].tolist() == [False, False, True, True, False, False]
+    assert keep[0].tolist() == [False, True, True, False, True, False]
+
+
+def test_topk_row_statistics_are_population_moments():
+    rng = np.random.default_rng(21)
+    s = rng.standard_normal((6, 37)) * 3.0 + 1.0
+    _, stats = oracle.topk_route(s, 0.6)
+    for i in range(6):
+        row = s[i].tolist()
+        assert abs(stats[i, 0] - statistics.fmean(row)) <= 1e-12 * 4
+        assert abs(stats[i, 1] - statistics.pstdev(row)) <= 1e-12 * 3
+
+
 def test_equal_rows_and_empty_routed_set():
     s = np.full((3, 8), 2.5)
     keep, _, _ = oracle.sol_route(s, 1.0)
