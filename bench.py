@@ -534,21 +534,27 @@ def oracle_sample(w, tau, n_route_heads, n_qblocks, seed=0):
             ref = oracle.route_head(q.float().numpy(), k.float().numpy(), tau, w.n_prefix)
             t_r += time.perf_counter() - a
             refs.append((ref, v.float().numpy()))
-        # attention units: n_qblocks query blocks spread over the routed heads
+        # attention units: n_qblocks query blocks spread over the routed heads. A call pays a
+        # per-head part (the centroid table, V in fp64) once, then a part per query block; the
+        # per-head part is timed alone (no query block) so that each part is scaled by its own count.
         per_head = max(1, min(w.nQB, n_qblocks // n_route_heads))
-        t_a, n_units = 0.0, 0
+        t_head, t_blocks, n_units = 0.0, 0.0, 0
         for ref, v in refs:
             blocks = sorted(int(x) for x in rng.choice(w.nQB, size=per_head, replace=False))
+            args = (ref["q8"], ref["q_scale"], ref["k8"], ref["k_scale"], v, ref["keep"], w.centroid_mode, 0.0)
             a = time.perf_counter()
-            oracle.sol_attention_head(ref["q8"], ref["q_scale"], ref["k8"], ref["k_scale"], v, ref["keep"],
-                                      w.centroid_mode, 0.0, q_blocks=blocks)
-            t_a += time.perf_counter() - a
+            oracle.sol_attention_head(*args, q_blocks=[])
+            b = time.perf_counter()
+            oracle.sol_attention_head(*args, q_blocks=blocks)
+            c = time.perf_counter()
+            t_head += b - a
+            t_blocks += max(0.0, (c - b) - (b - a))
             n_units += len(blocks)
     heads = w.B * w.H
-    est_s = t_r / n_route_heads * heads + t_a / n_units * heads * w.nQB
+    est_s = (t_r + t_head) / n_route_heads * heads + t_blocks / n_units * heads * w.nQB
     sample = (f"routing of {n_route_heads} head(s) (all {w.nQB} query-block rows) + attention of "
-              f"{n_units} query blocks ({per_head} per routed head), extrapolated by unit count to "
-              f"{heads} heads x {w.nQB} query blocks; 1 thread")
+              f"{n_units} query blocks ({per_head} per routed head); per-head and per-query-block parts "
+              f"timed apart and extrapolated by unit count to {heads} heads x {w.nQB} query blocks; 1 thread")
     return est_s * 1e3, sample, time.perf_counter() - t0
 
 
@@ -560,9 +566,9 @@ def run_reference(args, rank):
     tau = 1.0
     vals = []
     for _ in range(args.warmup):
-        oracle_sample(w, tau, 1, 2)
+        oracle_sample(w, tau, 1, 16)
     for s in range(args.steps):
-        v, sample, _ = oracle_sample(w, tau, 1, 2, seed=s)
+        v, sample, _ = oracle_sample(w, tau, 1, 16, seed=s)
         vals.append(v)
     value = float(np.mean(vals))
     line = {
