@@ -344,6 +344,7 @@ def roofline_numbers(w, work, r, peaks):
                        bytes=centroid_bytes(w)),
         mufu=mufu_bound(work, w, r["attn_ms"]),
         dense_equiv_tflops=round(w.dense_flops() / (r["ms"] * 1e-3) / 1e12, 2),
+        dense_equiv_frac=round(w.dense_flops() / (r["ms"] * 1e-3) / 1e12 / peak_eff, 4),
         kept_tflops=round(flops / (r["ms"] * 1e-3) / 1e12, 2),
     )
 
@@ -656,6 +657,7 @@ def main():
             sweep.append({"tau": tau, "ms_per_call": round(r2["ms"], 4), "route_ms": round(r2["route_ms"], 4),
                           "centroid_ms": round(r2["centroid_ms"], 4), "attn_ms": round(r2["attn_ms"], 4),
                           "sparsity": round(wk["sparsity"], 4), "dense_equiv_tflops": rf["dense_equiv_tflops"],
+                          "dense_equiv_frac_of_peak": rf["dense_equiv_frac"],
                           "kept_tflops": rf["kept_tflops"], "attn_roofline_frac": rf["attn"]["frac"]})
             bsva.check_status(s2.ws)
             del s2
@@ -697,6 +699,7 @@ def main():
                       "attention": round(r["attn_ms"], 4)},
         "sparsity": round(work["sparsity"], 4),
         "dense_equiv_tflops": roof["dense_equiv_tflops"] * world,
+        "dense_equiv_frac_of_peak": roof["dense_equiv_frac"],
         "kept_tflops": roof["kept_tflops"] * world,
         "roofline": roof["attn"],
         "route_roofline": roof["route"],

@@ -55,6 +55,8 @@ def test_roofline_numbers_are_consistent():
     assert abs(rf["kept_tflops"] - 2e12 / 1.25e-3 / 1e12) < 0.01
     assert abs(rf["route"]["achieved"] - bench.route_bytes(w) / 1e-4 / 1e9) < 0.1
     assert abs(rf["route"]["frac_of_spec"] * 8000.0 - rf["route"]["achieved"]) < 0.5
+    # dense-equivalent work over the whole call against the same effective tensor peak
+    assert abs(rf["dense_equiv_frac"] - w.dense_flops() / 1.25e-3 / 1e12 / rf["attn"]["peak"]) < 1e-3
 
 
 def test_centroid_bytes_and_mufu_bound_at_the_headline_shape():
