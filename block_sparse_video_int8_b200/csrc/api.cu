@@ -11,6 +11,7 @@
 #include <string>
 
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "common.cuh"
 
@@ -41,6 +42,17 @@ int ok() {
 int cuda_fail(cudaError_t e, const char* what) {
   return fail(BSVA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
+
+// An NVTX range over one entry point (its validation, descriptor encoding and
+// launches), named after the entry, so that a profiler timeline shows which
+// call issued which kernels. NVTX costs nothing measurable when no tool is attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define BSVA_RANGE(name) NvtxRange bsva_nvtx_range_(name)
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per device-side wait
 
@@ -198,6 +210,7 @@ size_t bsva_route_workspace_bytes(bsva_shape s) {
 
 int bsva_quantize_qk(bsva_shape s, const void* q, const void* k, int8_t* q8, float* q_scale, int8_t* k8,
                      float* k_scale, int32_t* q_pool, int32_t* k_pool, bsva_stream_t stream) {
+  BSVA_RANGE("bsva_quantize_qk");
   int rc;
   if ((rc = check_shape(s))) return rc;
   REQUIRE_PTR(q, 16); REQUIRE_PTR(k, 16); REQUIRE_PTR(q8, 16); REQUIRE_PTR(k8, 16);
@@ -214,6 +227,7 @@ int sparse_attn_route(bsva_shape s, const void* q, const void* k, double tau, in
                       float* k_scale, int32_t* q_pool, int32_t* k_pool, uint8_t* kept_mask, int32_t* kept_idx,
                       int32_t* kept_cnt, double* row_stats, void* workspace, size_t workspace_bytes,
                       bsva_stream_t stream) {
+  BSVA_RANGE("sparse_attn_route");
   int rc;
   if ((rc = check_shape(s))) return rc;
   if (std::isnan(tau)) return fail(BSVA_ERR_INVALID_ARG, "tau is NaN");
@@ -240,6 +254,7 @@ int sparse_attn_route_topk(bsva_shape s, const void* q, const void* k, double sp
                            float* q_scale, int8_t* k8, float* k_scale, int32_t* q_pool, int32_t* k_pool,
                            uint8_t* kept_mask, int32_t* kept_idx, int32_t* kept_cnt, double* row_stats,
                            void* workspace, size_t workspace_bytes, bsva_stream_t stream) {
+  BSVA_RANGE("sparse_attn_route_topk");
   int rc;
   if ((rc = check_shape(s))) return rc;
   if (!(sparsity >= 0.0 && sparsity <= 1.0)) return fail(BSVA_ERR_INVALID_ARG, "sparsity %g is not in [0, 1]", sparsity);
@@ -267,6 +282,7 @@ int sparse_attn_route_topk(bsva_shape s, const void* q, const void* k, double sp
 
 int bsva_build_lcsa_mask(int Lq, int Lk, int frame_tokens, int window_frames, int batch, uint8_t* mask,
                          bsva_stream_t stream) {
+  BSVA_RANGE("bsva_build_lcsa_mask");
   if (Lq < 1 || Lk < 1 || batch < 1) return fail(BSVA_ERR_INVALID_ARG, "Lq, Lk and batch must be >= 1");
   if (frame_tokens < 1) return fail(BSVA_ERR_INVALID_ARG, "frame_tokens = %d must be >= 1", frame_tokens);
   if (window_frames < 0) return fail(BSVA_ERR_INVALID_ARG, "window_frames = %d must be >= 0", window_frames);
@@ -327,6 +343,7 @@ extern "C" {
 
 int bsva_build_centroids(bsva_shape s, const int32_t* k_pool, const float* k_scale, const void* v,
                          int centroid_mode, void* workspace, size_t workspace_bytes, bsva_stream_t stream) {
+  BSVA_RANGE("bsva_build_centroids");
   int rc;
   if ((rc = check_centroid_args(s, k_pool, k_scale, v, centroid_mode))) return rc;
   const WsLayout L = ws_layout(s, centroid_mode);
@@ -342,6 +359,7 @@ int bsva_sparse_attn_core(bsva_shape s, const int8_t* q8, const float* q_scale, 
                           const float* k_scale, const void* v, const uint8_t* kept_mask, const int32_t* kept_idx,
                           const int32_t* kept_cnt, int centroid_mode, float softmax_scale, int out_dtype, void* out,
                           float* lse, void* workspace, size_t workspace_bytes, bsva_stream_t stream) {
+  BSVA_RANGE("bsva_sparse_attn_core");
   int rc;
   if ((rc = check_fwd_args(s, q8, q_scale, k8, k_scale, v, kept_mask, kept_idx, kept_cnt, centroid_mode,
                            softmax_scale, out_dtype, out, lse)))
@@ -358,6 +376,7 @@ int sparse_attn_fwd(bsva_shape s, const int8_t* q8, const float* q_scale, const 
                     const int32_t* k_pool, const void* v, const uint8_t* kept_mask, const int32_t* kept_idx,
                     const int32_t* kept_cnt, int centroid_mode, float softmax_scale, int out_dtype, void* out,
                     float* lse, void* workspace, size_t workspace_bytes, bsva_stream_t stream) {
+  BSVA_RANGE("sparse_attn_fwd");
   int rc;
   if ((rc = check_fwd_args(s, q8, q_scale, k8, k_scale, v, kept_mask, kept_idx, kept_cnt, centroid_mode,
                            softmax_scale, out_dtype, out, lse)))
@@ -377,6 +396,7 @@ int masked_block_attn_fwd(bsva_shape s, const int8_t* q8, const float* q_scale, 
                           const float* k_scale, const void* v, const uint8_t* block_mask, int mask_heads,
                           float softmax_scale, int out_dtype, void* out, float* lse, void* workspace,
                           size_t workspace_bytes, bsva_stream_t stream) {
+  BSVA_RANGE("masked_block_attn_fwd");
   int rc;
   if ((rc = check_shape(s))) return rc;
   if (mask_heads != 1 && mask_heads != s.H)
@@ -402,6 +422,7 @@ int masked_block_attn_fwd(bsva_shape s, const int8_t* q8, const float* q_scale, 
 }
 
 int bsva_quantize_v(bsva_shape s, const void* v, int8_t* v8, float* v_scale, bsva_stream_t stream) {
+  BSVA_RANGE("bsva_quantize_v");
   int rc;
   if ((rc = check_shape(s))) return rc;
   REQUIRE_PTR(v, 16); REQUIRE_PTR(v8, 16); REQUIRE_PTR(v_scale, 4);
@@ -417,6 +438,7 @@ int masked_block_attn_fwd_v8(bsva_shape s, const int8_t* q8, const float* q_scal
                              const uint8_t* block_mask, int mask_heads, float softmax_scale, int out_dtype,
                              void* out, float* lse, void* workspace, size_t workspace_bytes,
                              bsva_stream_t stream) {
+  BSVA_RANGE("masked_block_attn_fwd_v8");
   int rc;
   if ((rc = check_shape(s))) return rc;
   if (mask_heads != 1 && mask_heads != s.H)
@@ -464,6 +486,7 @@ int virtual_kv_residual_fwd(bsva_shape s, const int8_t* q8, const float* q_scale
                             const int* src_map, int n_virtual, int centroid_mode, float softmax_scale,
                             int out_dtype, void* out, float* lse, void* workspace, size_t workspace_bytes,
                             bsva_stream_t stream) {
+  BSVA_RANGE("virtual_kv_residual_fwd");
   int rc;
   if ((rc = check_shape(s))) return rc;
   if ((rc = check_virtual_geometry(slice_tokens, n_src_slices, centroid_mode))) return rc;
@@ -555,20 +578,62 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kNoAllocMaxDevices] = {};   // unique id of the context the address belongs to
 
-// Device address of the scratch array on the current device, looked up once
-// per device (host code cannot use the array's name as a device address).
+using PFN_ctxGetCurrent = CUresult (*)(CUcontext*);
+using PFN_ctxGetId = CUresult (*)(CUcontext, unsigned long long*);
+PFN_ctxGetCurrent g_ctx_get_current = nullptr;
+PFN_ctxGetId g_ctx_get_id = nullptr;
+std::once_flag g_ctx_once;
+
+// Unique id of the calling thread's current context, or 0 when none is current
+// yet (ids are never reused in a process, unlike context handles).
+int current_context_id(unsigned long long* id) {
+  std::call_once(g_ctx_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_get_current = reinterpret_cast<PFN_ctxGetCurrent>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_get_id = reinterpret_cast<PFN_ctxGetId>(fn);
+  });
+  if (!g_ctx_get_current || !g_ctx_get_id)
+    return fail(BSVA_ERR_CUDA, "cuCtxGetCurrent / cuCtxGetId are unavailable from the driver");
+  *id = 0;
+  CUcontext ctx = nullptr;
+  CUresult r = g_ctx_get_current(&ctx);
+  if (r != CUDA_SUCCESS) return fail(BSVA_ERR_CUDA, "cuCtxGetCurrent failed with %d", int(r));
+  if (ctx == nullptr) return BSVA_OK;
+  r = g_ctx_get_id(ctx, id);
+  if (r != CUDA_SUCCESS) return fail(BSVA_ERR_CUDA, "cuCtxGetId failed with %d", int(r));
+  return BSVA_OK;
+}
+
+// Device address of the scratch array in the current device's context. Host
+// code cannot use the array's name as a device address, so the address is
+// looked up with that device current: on the first call on a device, and
+// again whenever the device's context has been recreated (after
+// cudaDeviceReset the module can be loaded at another address). The lookup
+// itself creates the context when none is current yet.
 int noalloc_scratch(unsigned char** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(BSVA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  unsigned long long ctx = 0;
+  int rc = current_context_id(&ctx);
+  if (rc) return rc;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  if (ctx == 0 || g_noalloc_ptr[dev] == nullptr || g_noalloc_ctx[dev] != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+    if (ctx == 0 && (rc = current_context_id(&ctx))) return rc;   // the lookup made the context current
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = ctx;
   }
   *out = static_cast<unsigned char*>(g_noalloc_ptr[dev]);
   return BSVA_OK;
@@ -580,6 +645,7 @@ extern "C" int masked_block_attn_fwd_noalloc(bsva_shape s, const int8_t* q8, con
                                              const float* k_scale, const void* v, const uint8_t* block_mask,
                                              int mask_heads, float softmax_scale, int out_dtype, void* out,
                                              float* lse, bsva_stream_t stream) {
+  BSVA_RANGE("masked_block_attn_fwd_noalloc");
   int rc;
   if ((rc = check_shape(s))) return rc;
   if (mask_heads != 1 && mask_heads != s.H)

@@ -312,8 +312,9 @@ int virtual_kv_residual_fwd(bsva_shape s, const int8_t* q8, const float* q_scale
  * Limits: B*H*nQB <= 65,536 and B*H*nQB*nKB <= 2,097,152; a larger shape
  * returns BSVA_ERR_WORKSPACE and launches nothing.
  * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture. Every call shares the one array, which keeps the
+ * (cudaGetSymbolAddress) with that device current, and so does the first call
+ * after the device's context has been recreated (cudaDeviceReset); make such
+ * a first call before any stream capture. Every call shares the one array, which keeps the
  * last call's contents: calls whose GPU work overlaps (two streams, two host
  * threads) race on it, so the caller must serialise them. A device-side wait
  * that runs out is recorded in the array's status word, which this entry

@@ -1,15 +1,20 @@
 """Mutation check of the CPU oracle's pins (run by hand; pytest does not collect it).
 
-Each entry plants one plausible mistake in ``oracle/`` (a dropped term, a wrong
-index or bound, a flipped comparison or sign, another rounding), runs the
-oracle's CPU pins (``tests/test_oracle_*.py``) and restores the file. A pin
-set is adequate when every mistake is caught ("KILLED").
+Each entry plants one plausible mistake (a dropped term, a wrong index or
+bound, a flipped comparison or sign, another rounding) in a temporary copy of
+``oracle/`` and runs the oracle's CPU pins (``tests/test_oracle_*.py``) on that
+copy; the tracked files are never written. A mistake counts as caught
+("KILLED") only when the pins ran and at least one failed (pytest exit 1); a
+collection error or a timeout is reported as an error. A pin set is adequate
+when every mistake is caught.
 
     python tests/oracle_mutations.py
 """
 import os
+import shutil
 import subprocess
 import sys
+import tempfile
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PINS = ["tests/test_oracle_quant.py", "tests/test_oracle_route.py", "tests/test_oracle_attention.py"]
@@ -60,27 +65,48 @@ M = [
 ]
 
 
+def _copy_tree(dst: str) -> None:
+    """The oracle, its pins and their imports, copied so that mutations never touch tracked files."""
+    for d in ("oracle", "tests", "workloads"):
+        shutil.copytree(os.path.join(ROOT, d), os.path.join(dst, d),
+                        ignore=shutil.ignore_patterns("__pycache__", "*.pyc"))
+
+
 def main() -> int:
-    survivors = []
-    for f, old, new in M:
-        path = os.path.join(ROOT, f)
-        src = open(path).read()
-        if src.count(old) != 1:
-            print("NO MATCH", f, old[:60])
-            survivors.append((f, new))
-            continue
-        open(path, "w").write(src.replace(old, new))
-        try:
-            r = subprocess.run([sys.executable, "-m", "pytest", *PINS, "-x", "-q", "-p", "no:cacheprovider"],
-                               cwd=ROOT, capture_output=True, text=True, timeout=900)
-            killed = r.returncode != 0
-        finally:
-            open(path, "w").write(src)
-        print("KILLED  " if killed else "SURVIVED", f, "|", " ".join(new.split())[:90], flush=True)
-        if not killed:
-            survivors.append((f, new))
-    print(f"{len(M) - len(survivors)} of {len(M)} mutations caught")
-    return 1 if survivors else 0
+    survivors, errors = [], []
+    with tempfile.TemporaryDirectory(prefix="oracle_mut_") as tmp:
+        _copy_tree(tmp)
+        for f, old, new in M:
+            path = os.path.join(tmp, f)
+            src = open(path).read()
+            if src.count(old) != 1:
+                print("NO MATCH", f, old[:60])
+                errors.append((f, new))
+                continue
+            open(path, "w").write(src.replace(old, new))
+            try:
+                r = subprocess.run([sys.executable, "-m", "pytest", *PINS, "-x", "-q", "-p", "no:cacheprovider"],
+                                   cwd=tmp, capture_output=True, text=True, timeout=900)
+                rc = r.returncode
+            except subprocess.TimeoutExpired:
+                rc = None
+            finally:
+                open(path, "w").write(src)
+            # pytest exits 1 when tests ran and some failed: only that counts as caught. Exit 2-4
+            # (interrupted, internal error, usage or collection error) and a timeout are errors.
+            if rc == 1:
+                verdict = "KILLED  "
+            elif rc == 0:
+                verdict = "SURVIVED"
+                survivors.append((f, new))
+            else:
+                verdict = f"ERROR({rc})"
+                errors.append((f, new))
+            print(verdict, f, "|", " ".join(new.split())[:90], flush=True)
+    caught = len(M) - len(survivors) - len(errors)
+    print(f"{caught} of {len(M)} mutations caught by a failing pin; {len(survivors)} survived; "
+          f"{len(errors)} errors (no match, collection error or timeout)")
+    return 1 if survivors or errors else 0
 
 
 if __name__ == "__main__":

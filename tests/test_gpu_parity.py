@@ -13,8 +13,8 @@ import torch
 
 import oracle
 import workloads
-from parity import (Report, assert_within, compare_rows, head_np, inputs, masked_parity, masked_parity_v8,
-                    q_rows, sol_parity, to_np, topk_parity, virtual_parity)
+from parity import (Report, assert_band_small, assert_within, compare_rows, head_np, inputs, lcsa_input_mask, masked_parity,
+                    masked_parity_v8, q_rows, sol_parity, to_np, topk_parity, virtual_parity)
 
 pytestmark = pytest.mark.gpu
 
@@ -42,6 +42,72 @@ def test_sol_high_tau_centroid_heavy(gpu_lib):
     w = workloads.get("ragged_pe_2x32")
     route, out, lse, rep = sol_parity(gpu_lib, w, 2.5)
     assert_within(rep, "tau=2.5")
+
+
+def _zero_blocks(w):
+    """The workload's inputs with an all-zero query block (rows 128..255 of head (0, 0)) and an
+    all-zero key block (rows 64..127 of heads (0, 0) and (0, 1)): scale 0, every code 0."""
+    Q, K, V = workloads.batch_qkv(w)
+    Q[0, 0, 128:256] = 0
+    K[0, 0, 64:128] = 0
+    K[0, 1, 64:128] = 0
+    return Q, K, V
+
+
+@pytest.mark.parametrize("name,tau", [("ragged_pe", 1.0), ("ragged_pe", -math.inf), ("ragged_pe_2x32", 1.0),
+                                      ("ragged_pe_2x32", -1.0)])
+def test_sol_zero_q_and_k_blocks(gpu_lib, name, tau):
+    # A zero Q block has scale 0: its logits are all 0 (every routed score ties, so the row keeps
+    # every block) and the kernel's logit factor is 0 for every tile. A zero K block has scale 0:
+    # its score is 0, and it enters exactly (factor 0) when kept, or through a centroid of key 0
+    # when skipped.
+    w = workloads.get(name)
+    qkv = _zero_blocks(w)
+    route, out, lse, rep = sol_parity(gpu_lib, w, tau, qkv=qkv)
+    assert_within(rep, f"{name} zero blocks tau={tau}")
+    assert float(route.q_scale[0, 0, 1]) == 0.0 and float(route.k_scale[0, 0, 1]) == 0.0
+    assert bool((route.kept_mask[0, 0, 1] == 1).all())          # the zero query block keeps every block
+    print(f"{name} zero blocks tau={tau}: {rep}")
+
+
+def test_masked_zero_q_and_k_blocks(gpu_lib):
+    w = workloads.get("cross")
+    qkv = _zero_blocks(w)
+    m = np.ones((w.B, w.H, w.nQB, w.nLK), np.uint8)
+    m[0, 0, 2, :] = 0
+    out, lse, rep = masked_parity(gpu_lib, w, torch.from_numpy(m), qkv=qkv)
+    assert_within(rep, "mask entry zero blocks")
+
+
+@pytest.mark.parametrize("mag", [1e-35, 3e-38])
+def test_sol_tiny_scales_take_the_exact_division(gpu_lib, mag):
+    # A block whose amax puts s = fl(amax/127) below 2^-120 (1e-35: a normal scale near 2^-121;
+    # 3e-38: a subnormal scale) is quantised by IEEE division, element by element.
+    w = workloads.get("ragged_pe")
+    Q, K, V = workloads.batch_qkv(w)
+    K[0, 0, 128:192] = (K[0, 0, 128:192].float() * mag).to(torch.bfloat16)
+    Q[1, 2, 256:384] = (Q[1, 2, 256:384].float() * mag).to(torch.bfloat16)
+    K[1, 2, 960:1000] = (K[1, 2, 960:1000].float() * mag).to(torch.bfloat16)    # the 40-row tail block
+    route, out, lse, rep = sol_parity(gpu_lib, w, 1.0, qkv=(Q, K, V))
+    assert_within(rep, f"tiny scales {mag}")
+    s = float(route.k_scale[0, 0, 2])
+    assert 0.0 < s < 2.0 ** -120
+
+
+def test_sol_all_equal_routed_row_keeps_every_block(gpu_lib):
+    # Identical keys make every routed score of a row equal (Lk = 2048 is a whole number of key
+    # blocks, so no tail block differs): max == min, and the row keeps every block whatever tau
+    # (T = -inf in the row statistics; sigma is 0 up to the rounding of the mean).
+    w = workloads.get("tiny")
+    Q, K, V = workloads.batch_qkv(w)
+    K = K[:, :, :1, :].expand_as(K).contiguous()
+    for tau in (1.0, 1.5):
+        route, out, lse, rep = sol_parity(gpu_lib, w, tau, qkv=(Q, K, V))
+        assert_within(rep, f"all-equal rows tau={tau}")
+        assert bool((route.kept_mask == 1).all())
+        st = route.row_stats.cpu().numpy()
+        assert np.isneginf(st[..., 2]).all()
+        assert (st[..., 1] <= 1e-12 * np.abs(st[..., 0])).all()
 
 
 @pytest.mark.parametrize("name,sparsity", [("ragged_pe", 0.75), ("ragged_pe_2x32", 0.5), ("ragged_d64", 0.9),
@@ -74,7 +140,7 @@ def test_topk_ties_broken_by_index(gpu_lib):
 
 def test_masked_small_lcsa(gpu_lib):
     w = workloads.get("lcsa_small")
-    _, _, rep = masked_parity(gpu_lib, w, workloads.block_mask(w))
+    _, _, rep = masked_parity(gpu_lib, w, lcsa_input_mask(w))
     assert_within(rep, "lcsa_small")
 
 
@@ -101,7 +167,7 @@ def test_masked_small_lcsa_device_mask(gpu_lib):
 
 def test_masked_v8_small_lcsa(gpu_lib):
     w = workloads.get("lcsa_small")
-    _, _, rep = masked_parity_v8(gpu_lib, w, workloads.block_mask(w))
+    _, _, rep = masked_parity_v8(gpu_lib, w, lcsa_input_mask(w))
     assert_within(rep, "lcsa_small INT8 V")
 
 
@@ -195,7 +261,7 @@ def _sample_blocks(nQB, n_extra=4, seed=0):
 def test_full_lcsa_v8(gpu_lib):
     w = workloads.get("lcsa")
     heads = [(0, 0), (0, w.H - 1)]
-    _, _, rep = masked_parity_v8(gpu_lib, w, workloads.block_mask(w), heads=heads,
+    _, _, rep = masked_parity_v8(gpu_lib, w, lcsa_input_mask(w), heads=heads,
                                  q_blocks=_sample_blocks(w.nQB))
     assert_within(rep, "lcsa full INT8 V")
 
@@ -213,7 +279,7 @@ def test_full_virtual_kv(gpu_lib):
 def test_full_lcsa(gpu_lib):
     w = workloads.get("lcsa")
     heads = [(0, 0), (0, w.H - 1)]
-    _, _, rep = masked_parity(gpu_lib, w, workloads.block_mask(w), heads=heads,
+    _, _, rep = masked_parity(gpu_lib, w, lcsa_input_mask(w), heads=heads,
                               q_blocks=_sample_blocks(w.nQB))
     assert_within(rep, "lcsa full")
 
@@ -221,20 +287,24 @@ def test_full_lcsa(gpu_lib):
 @pytest.mark.slow
 @pytest.mark.parametrize("name,sparsity", [("wan14b", 0.75), ("h3", 0.75)])
 def test_full_topk(gpu_lib, name, sparsity):
+    # routing and quantisation of every head bit for bit; outputs on heads {0, H-1}
     w = workloads.get(name)
-    heads = [(0, 0), (0, w.H - 1)]
-    _, _, _, rep = topk_parity(gpu_lib, w, sparsity, heads=heads, q_blocks=_sample_blocks(w.nQB))
+    _, _, _, rep = topk_parity(gpu_lib, w, sparsity, attn_heads=[(0, 0), (0, w.H - 1)],
+                               q_blocks=_sample_blocks(w.nQB))
     print(f"{name} top-k sparsity={sparsity}: {rep}")
     assert_within(rep, f"{name} top-k sparsity={sparsity}")
+    assert rep.blocks == w.B * w.H * w.nQB * w.nKB
 
 
 @pytest.mark.slow
 @pytest.mark.parametrize("name,tau", [("wan13b", 1.0), ("wan14b", 0.5), ("wan14b", 1.0), ("wan14b", 1.5),
                                       ("h3", 1.0)])
 def test_full_sol(gpu_lib, name, tau):
+    # routing and quantisation of every head bit for bit (band excepted and bounded); outputs on
+    # heads {0, H-1} over sampled query blocks
     w = workloads.get(name)
-    heads = [(0, 0), (0, w.H - 1)]
-    _, _, _, rep = sol_parity(gpu_lib, w, tau, heads=heads, q_blocks=_sample_blocks(w.nQB))
+    _, _, _, rep = sol_parity(gpu_lib, w, tau, attn_heads=[(0, 0), (0, w.H - 1)], q_blocks=_sample_blocks(w.nQB))
     print(f"{name} tau={tau}: {rep}")
     assert_within(rep, f"{name} tau={tau}")
-    assert rep.band_mismatch <= max(2, rep.band)
+    assert rep.blocks == w.B * w.H * w.nQB * w.nKB
+    assert_band_small(rep, f"{name} tau={tau}")

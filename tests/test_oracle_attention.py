@@ -100,7 +100,7 @@ def test_identical_token_block_same_kept_or_skipped(mode):
 def test_mask_entry_matches_token_level_masked_dense():
     w, q, k, v = _head("lcsa_small")
     r = oracle.route_head(q, k, -math.inf)
-    logical = workloads.block_mask(w)[0, 0].numpy()
+    logical = oracle.lcsa_mask(w.Lq, w.Lk, w.frame_tokens, w.lcsa_window)
     allowed = oracle.physical_allowed(logical, w.nKB)
     O, lse = oracle.masked_attention_head(r["q8"], r["q_scale"], r["k8"], r["k_scale"], v, allowed)
     Lq, Lk = w.Lq, w.Lk

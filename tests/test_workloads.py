@@ -5,22 +5,6 @@ import torch
 import workloads
 
 
-def test_lcsa_mask_density_is_21_over_64():
-    w = workloads.get("lcsa")
-    m = workloads.block_mask(w)
-    assert tuple(m.shape) == (1, 1, 96, 96)
-    assert int(m.sum()) * 64 == 21 * 96 * 96
-
-
-def test_lcsa_window_rule():
-    m = workloads.lcsa_block_mask(128 * 30, 128 * 30, 384, 2)   # 3 blocks per frame
-    for i in range(30):
-        fq = i // 3
-        for x in range(30):
-            fk = x // 3
-            assert bool(m[i, x]) == (fq - 2 <= fk <= fq)
-
-
 def test_heads_reproducible_and_independent():
     w = workloads.get("ragged_pe")
     a = workloads.head_qkv(w, 1, 2)

@@ -7,16 +7,20 @@ device): its kept-block lists live in a scratch array built into the library.
 This test runs two calls in a row with different inputs and masks, so that a
 result left over in the shared scratch from the first call would show up in
 the second, and checks each against ``masked_block_attn_fwd`` with a caller
-workspace, within the tolerances the parity tests use. It is collected last
-and needs no state from other tests.
+workspace and against the fp64 oracle (every head, every query block), within
+the tolerances the parity tests use. It is collected last and needs no state
+from other tests.
 """
 import ctypes
+import math
 
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import workloads
+from parity import Report, assert_within, compare_rows, head_np, lcsa_input_mask, q_rows, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -44,6 +48,23 @@ def _check(got, ref):
     assert float(err.norm() / r.norm()) <= REL_L2
 
 
+def _check_oracle(w, out, lse, mask, what):
+    """Every head and query block of one call against the oracle's masked attention."""
+    rep = Report()
+    Hm = mask.shape[1]
+    m = mask.cpu().numpy()
+    for b in range(w.B):
+        for h in range(w.H):
+            q, k, v = head_np(w, b, h)
+            ref = oracle.route_head(q, k, -math.inf, 0)
+            allowed = oracle.physical_allowed(m[b, h % Hm], w.nKB)
+            O_ref, lse_ref = oracle.masked_attention_head(ref["q8"], ref["q_scale"], ref["k8"], ref["k_scale"], v,
+                                                          allowed)
+            compare_rows(to_np(out[b, h].float()), to_np(lse[b, h]), O_ref, lse_ref,
+                         q_rows(w.Lq, range(w.nQB)), rep)
+    assert_within(rep, what)
+
+
 def test_noalloc_mask_entry_matches_workspace_entry_twice(gpu_lib):
     bsva = gpu_lib
     lib = bsva.load()
@@ -51,7 +72,7 @@ def test_noalloc_mask_entry_matches_workspace_entry_twice(gpu_lib):
     w = workloads.get("lcsa_small")
     Q, K, V = [x.cuda() for x in workloads.batch_qkv(w)]
     qk = bsva.quantize_qk(Q, K)
-    mask1 = workloads.block_mask(w).cuda()
+    mask1 = lcsa_input_mask(w).cuda()
     ref1, rl1 = bsva.masked_block_attn_fwd(qk["q8"], qk["q_scale"], qk["k8"], qk["k_scale"], V, mask1,
                                            with_lse=True, out_dtype=torch.float32)
     got1, gl1 = _noalloc(lib, bsva, qk, V, mask1)
@@ -69,6 +90,8 @@ def test_noalloc_mask_entry_matches_workspace_entry_twice(gpu_lib):
     torch.cuda.synchronize()
     _check(got1, ref1)
     _check(got2, ref2)
+    _check_oracle(w, got1, gl1, mask1, "no-alloc call 1 vs oracle")
+    _check_oracle(w2, got2, gl2, mask2, "no-alloc call 2 vs oracle")
     fin = torch.isfinite(rl2)
     assert torch.equal(fin, torch.isfinite(gl2))
     assert float((gl2[fin] - rl2[fin]).abs().max()) <= 1e-3

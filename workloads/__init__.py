@@ -1,9 +1,11 @@
 """Seeded synthetic inputs for block-sparse INT8 video attention.
 
 This module is the one piece shared by the CPU oracle (``oracle/``) and the
-CUDA path (``block_sparse_video_int8_b200``): it draws Q, K, V and the LCSA
-logical block mask, and holds none of the method's arithmetic (no
-quantisation, scoring, routing or attention).
+CUDA path (``block_sparse_video_int8_b200``): it draws Q, K, V and records
+each workload's geometry (frame size and window of the LCSA mask), and holds
+none of the method's arithmetic (no quantisation, scoring, routing,
+attention, and no mask rule: tests build the LCSA mask input with the oracle,
+the bench with the library's device builder).
 
 Workload shapes follow the video-diffusion settings the source pages name:
 Wan-style self-attention over a frame-major latent video
@@ -36,8 +38,7 @@ import numpy as np
 import torch
 
 __all__ = [
-    "Workload", "WORKLOADS", "get", "head_qkv", "batch_qkv", "block_mask",
-    "lcsa_block_mask", "pe_table", "W_SEED", "source_kv",
+    "Workload", "WORKLOADS", "get", "head_qkv", "batch_qkv", "pe_table", "W_SEED", "source_kv",
 ]
 
 W_SEED = 7
@@ -237,24 +238,3 @@ def batch_qkv(w: Workload, heads=None, device="cpu"):
         K[b, h].copy_(k)
         V[b, h].copy_(v)
     return Q, K, V
-
-
-def lcsa_block_mask(Lq: int, Lk: int, frame_tokens: int, window: int = 2) -> np.ndarray:
-    """FlashVSR-style local causal mask on logical 128x128 blocks, uint8 [nQB, nLK].
-
-    A logical block x lies in frame floor(128*x / frame_tokens); key block x_k
-    is allowed for query block x_q iff its frame is in [f_q - window, f_q].
-    """
-    nq, nk = -(-Lq // 128), -(-Lk // 128)
-    fq = (128 * np.arange(nq)) // frame_tokens
-    fk = (128 * np.arange(nk)) // frame_tokens
-    allowed = (fk[None, :] <= fq[:, None]) & (fk[None, :] >= fq[:, None] - window)
-    return allowed.astype(np.uint8)
-
-
-def block_mask(w: Workload) -> torch.Tensor:
-    """Logical mask of a mask-entry workload, uint8 [B, 1, nQB, nLK] (shared by heads)."""
-    if w.mask != "lcsa":
-        raise ValueError(f"workload {w.name} has no block mask")
-    m = lcsa_block_mask(w.Lq, w.Lk, w.frame_tokens, w.lcsa_window)
-    return torch.from_numpy(np.broadcast_to(m, (w.B, 1) + m.shape).copy())
