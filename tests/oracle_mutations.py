@@ -17,7 +17,8 @@ import sys
 import tempfile
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-PINS = ["tests/test_oracle_quant.py", "tests/test_oracle_route.py", "tests/test_oracle_attention.py"]
+PINS = ["tests/test_oracle_quant.py", "tests/test_oracle_route.py", "tests/test_oracle_attention.py",
+        "tests/test_oracle_kv_cache.py"]
 
 M = [
  ('oracle/quant.py', 's = np.float32(amax / np.float32(127.0))', 's = np.float32(amax / np.float32(128.0))'),
@@ -62,6 +63,13 @@ M = [
  ('oracle/attention.py', 'virtual = [grp for s in src_map for', 'virtual = [grp for s in sorted(set(src_map)) for'),
  ('oracle/attention.py', 'for j in range(s * bps, (s + 1) * bps)', 'for j in range(s * bps, (s + 1) * bps - 1)'),
  ('oracle/attention.py', 'for j in range(s * bps, (s + 1) * bps) for grp', 'for j in range((n_src - 1 - s) * bps, (n_src - s) * bps) for grp'),
+ ('oracle/kv_cache.py', 'for t0, t1 in block_rows(k.shape[0], SLAB_ROWS):', 'for t0, t1 in block_rows(k.shape[0], 64):'),
+ ('oracle/kv_cache.py', 'self.slabs.pop(0)', 'self.slabs.pop()'),
+ ('oracle/kv_cache.py', 'logits.append((float(q_scale[i]) * float(s["k_scale"][b]) * scale) * dots)', 'logits.append((float(q_scale[i]) * float(s["k_scale"][0]) * scale) * dots)'),
+ ('oracle/kv_cache.py', 'values.append(s["v8"][t0:t1].astype(np.float64) * float(s["v_scale"][b]))', 'values.append(s["v8"][t0:t1].astype(np.float64))'),
+ ('oracle/kv_cache.py', '            if not mask[i, x]:', '            if not mask[i, len(cache.slabs) - 1 - x]:'),
+ ('oracle/kv_cache.py', 'v8, vs = quantize_blocks(v[t0:t1], K_ROWS)', 'v8, vs = quantize_blocks(v[t0:t1], Q_ROWS)'),
+ ('oracle/kv_cache.py', 'while len(self.slabs) > self.capacity:', 'while len(self.slabs) > self.capacity + 1:'),
 ]
 
 
