@@ -556,6 +556,69 @@ def lcsa_measure(bsva, steps, warmup, dist, rank, world, int8_v=False):
             "dense_equiv_tflops": round(w0.dense_flops() / (ms * 1e-3) / 1e12, 2)}
 
 
+def kv_cache_measure(bsva, steps, warmup, dist, rank, world):
+    """The INT8 streaming K/V cache in 128-row slabs at the LCSA shape (B=1, H=12, d=128, frames of
+    32x48 = 1536 tokens = 12 slabs, window [f-2, f]): (1) the whole 8-frame window read through the
+    cache's ring (filled with 8 one-frame chunks after 3 earlier ones were evicted, so the ring wraps),
+    all 12288 queries under the LCSA mask built on the device; (2) one streaming step: append the next
+    frame (evicting the oldest), quantise its 1536 queries and attend to the 3 newest frames."""
+    w0 = workloads.get("lcsa")
+    w, heads = shard(w0, rank, world)
+    Q, K, V = [x.cuda() for x in shard_qkv(w0, heads)]
+    F = w.frame_tokens
+    n_frames = w.Lk // F
+    spf = F // 128                                      # slabs per frame
+    cache = bsva.KVCache(w.B, w.H, w.d, n_frames * spf)
+    for f in range(3):                                  # three frames that the window evicts again
+        cache.append(K[:, :, f * F:(f + 1) * F].contiguous(), V[:, :, f * F:(f + 1) * F].contiguous())
+    for f in range(n_frames):
+        cache.append(K[:, :, f * F:(f + 1) * F].contiguous(), V[:, :, f * F:(f + 1) * F].contiguous())
+    torch.cuda.synchronize()
+    mask = bsva.build_lcsa_mask(w.Lq, w.Lk, F, w.lcsa_window, batch=w.B)     # [B, 1, nQB, 96]: slab x = block x
+    qq = bsva.quantize_q(Q)
+    ws = torch.zeros(cache.workspace_bytes(w.Lq), dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(Q)
+
+    def full():
+        bsva.quantize_q(Q, out=qq)
+        cache.attend(qq, mask, workspace=ws, out=out)
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    ms_full = _timed_calls(full, steps, warmup, dist, flush=flush)
+    # streaming: a ring of 3 frames; each step appends the next frame and attends its queries
+    ring = bsva.KVCache(w.B, w.H, w.d, 3 * spf)
+    for f in range(3):
+        ring.append(K[:, :, f * F:(f + 1) * F].contiguous(), V[:, :, f * F:(f + 1) * F].contiguous())
+    chunks = [(K[:, :, f * F:(f + 1) * F].contiguous(), V[:, :, f * F:(f + 1) * F].contiguous(),
+               Q[:, :, f * F:(f + 1) * F].contiguous()) for f in range(n_frames)]
+    smask = torch.ones((w.B, 1, spf, 3 * spf), dtype=torch.uint8, device="cuda")
+    sq = bsva.quantize_q(chunks[0][2])
+    sws = torch.zeros(ring.workspace_bytes(F), dtype=torch.uint8, device="cuda")
+    sout = torch.empty_like(chunks[0][2])
+    state = {"f": 0}
+
+    def stream_step():
+        k, v, q = chunks[state["f"] % n_frames]
+        state["f"] += 1
+        ring.append(k, v)
+        bsva.quantize_q(q, out=sq)
+        ring.attend(sq, smask, workspace=sws, out=sout)
+
+    ms_step = _timed_calls(stream_step, steps, warmup, dist, flush=flush)
+    del flush
+    bsva.check_status(ws)
+    bsva.check_status(sws)
+    allowed = int(mask.sum().item()) * 128 * 128 * w0.H * w0.B
+    return {"workload": "lcsa through the INT8 streaming cache: B=1 H=12 d=128, 128-row slabs, frames of 32x48",
+            "full_window": {"what": "quantise 12288 queries + mask attention over the 96 live slabs of a wrapped "
+                                    "ring, INT8 K and V read in place", "ms_per_call": round(ms_full, 4),
+                            "kept_tflops": round(4.0 * w.d * allowed / (ms_full * 1e-3) / 1e12, 2)},
+            "streaming_step": {"what": "append one frame (1536 tokens, 12 slabs; evicts the oldest) + quantise its "
+                                       "queries + attention to the 3 newest frames (36 slabs)",
+                               "ms_per_step": round(ms_step, 4)},
+            "l2": "256 MB written between calls, outside the timed events"}
+
+
 def virtual_work(w, n_virtual):
     """Algorithmic FLOPs of one residual virtual K/V call: every physical pair exact, plus one
     centroid logit and one centroid value row per virtual group and query row."""
@@ -852,6 +915,7 @@ def main():
         extra["lcsa_mask_entry"] = lcsa_measure(bsva, max(5, args.steps // 4), 3, dist, rank, world)
         extra["lcsa_mask_entry_int8_v"] = lcsa_measure(bsva, max(5, args.steps // 4), 3, dist, rank, world,
                                                        int8_v=True)
+        extra["int8_kv_cache"] = kv_cache_measure(bsva, max(5, args.steps // 4), 3, dist, rank, world)
         extra["virtual_kv_residual"] = virtual_kv_measure(bsva, max(5, args.steps // 4), 3, dist, rank, world,
                                                           peaks)
     e2e = None

@@ -16,6 +16,10 @@ Entry points (same names as the C ABI):
 * ``quantize_v(v)``, ``masked_block_attn_fwd_v8(...)`` the mask entry on an INT8 V
 * ``virtual_kv_residual_fwd(qk, v, slice_tokens, src_map)`` residual virtual K/V:
   physical keys exact, each added virtual slice as centroid terms
+* ``quantize_q(q)``                          per-block INT8 Q alone
+* ``KVCache(B, H, d, n_slots)``              the INT8 streaming K/V cache in 128-row slabs:
+  ``append(k, v)`` (``bsva_kv_cache_append``) and ``attend(qq, mask)``
+  (``masked_block_attn_fwd_kvcache``)
 """
 from __future__ import annotations
 
@@ -31,9 +35,10 @@ __all__ = [
     "sparse_attn_route_topk", "build_lcsa_mask", "quantize_v", "masked_block_attn_fwd_v8", "sparse_attn_fwd",
     "masked_block_attn_fwd", "check_status", "selftest_timeout", "new_workspace",
     "build_centroids", "sparse_attn_core", "virtual_kv_workspace_bytes", "virtual_kv_residual_fwd",
+    "quantize_q", "KVCache",
 ]
 
-ABI_VERSION = 3
+ABI_VERSION = 4
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
 
@@ -52,6 +57,14 @@ class BsvaError(RuntimeError):
 class Shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("Lq", ctypes.c_int),
                 ("Lk", ctypes.c_int), ("d", ctypes.c_int), ("n_prefix", ctypes.c_int)]
+
+
+class KVCacheStruct(ctypes.Structure):
+    """``bsva_kv_cache``: geometry, device buffers, and the ring state the library updates."""
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int), ("n_slots", ctypes.c_int),
+                ("k8", ctypes.c_void_p), ("k_scale", ctypes.c_void_p), ("v8", ctypes.c_void_p),
+                ("v_scale", ctypes.c_void_p), ("slab_rows", ctypes.c_void_p),
+                ("first", ctypes.c_int), ("count", ctypes.c_int)]
 
 
 def lib_path() -> str:
@@ -87,6 +100,12 @@ _SIGS = {
                                                 ctypes.c_float, ctypes.c_int, _P, _P, _P, ctypes.c_size_t,
                                                 _P]),
     "bsva_selftest_timeout": (ctypes.c_int, [_P, ctypes.c_size_t, ctypes.c_longlong, _P]),
+    "bsva_quantize_q": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P]),
+    "bsva_kv_cache_append": (ctypes.c_int, [ctypes.POINTER(KVCacheStruct), _P, _P, ctypes.c_int, _P]),
+    "bsva_kv_cache_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(KVCacheStruct), ctypes.c_int]),
+    "masked_block_attn_fwd_kvcache": (ctypes.c_int, [ctypes.POINTER(KVCacheStruct), ctypes.c_int, _P, _P, _P,
+                                                     ctypes.c_int, ctypes.c_float, ctypes.c_int, _P, _P, _P,
+                                                     ctypes.c_size_t, _P]),
     "bsva_virtual_kv_workspace_bytes": (ctypes.c_size_t, [Shape, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     "virtual_kv_residual_fwd": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_int, _P, _P, _P,
                                                ctypes.POINTER(ctypes.c_int), ctypes.c_int, ctypes.c_int,
@@ -479,3 +498,84 @@ def selftest_timeout(workspace: torch.Tensor, limit_ns: int, stream=None):
     """Launch the bounded-wait self test (a wait that is meant to run out)."""
     _check(load().bsva_selftest_timeout(_ptr(workspace), workspace.numel(), int(limit_ns),
                                         _stream(stream)))
+
+
+def quantize_q(q: torch.Tensor, out: dict | None = None, stream=None) -> dict:
+    """Per-128-row-block INT8 Q with scales and sum-pools (C ABI ``bsva_quantize_q``)."""
+    lib = load()
+    _need(q, torch.bfloat16, None, "q")
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, Lq, d]")
+    B, H, Lq, d = q.shape
+    nQB = -(-Lq // 128)
+    o = out or dict(q8=torch.empty(q.shape, dtype=torch.int8, device=q.device),
+                    q_scale=torch.empty((B, H, nQB), dtype=torch.float32, device=q.device),
+                    q_pool=torch.empty((B, H, nQB, d), dtype=torch.int32, device=q.device))
+    _check(lib.bsva_quantize_q(Shape(B, H, Lq, Lq, d, 0), _ptr(q), _ptr(o["q8"]), _ptr(o["q_scale"]),
+                               _ptr(o["q_pool"]), _stream(stream)))
+    return o
+
+
+class KVCache:
+    """The INT8 streaming K/V cache in 128-row slabs (C ABI ``bsva_kv_cache``).
+
+    The device buffers are torch tensors owned by this object; ``append`` and ``attend``
+    call the library, which keeps the ring state (oldest slot, live slabs) in the struct."""
+
+    def __init__(self, B: int, H: int, d: int, n_slots: int, device=None):
+        dev = device or "cuda"
+        rows = n_slots * 128
+        self.k8 = torch.zeros((B, H, rows, d), dtype=torch.int8, device=dev)
+        self.v8 = torch.zeros((B, H, rows, d), dtype=torch.int8, device=dev)
+        self.k_scale = torch.zeros((B, H, 2 * n_slots), dtype=torch.float32, device=dev)
+        self.v_scale = torch.zeros((B, H, 2 * n_slots), dtype=torch.float32, device=dev)
+        self.slab_rows = torch.zeros((n_slots,), dtype=torch.int32, device=dev)
+        self.c = KVCacheStruct(B, H, d, n_slots, self.k8.data_ptr(), self.k_scale.data_ptr(), self.v8.data_ptr(),
+                               self.v_scale.data_ptr(), self.slab_rows.data_ptr(), 0, 0)
+
+    @property
+    def first(self) -> int:
+        return self.c.first
+
+    @property
+    def count(self) -> int:
+        return self.c.count
+
+    def append(self, k: torch.Tensor, v: torch.Tensor, stream=None):
+        """Quantise a chunk of new tokens (bf16 [B, H, Lc, d]) into the next slabs, evicting the oldest."""
+        c = self.c
+        _need(k, torch.bfloat16, None, "k")
+        if k.dim() != 4 or tuple(k.shape[:2]) != (c.B, c.H) or k.shape[3] != c.d:
+            raise ValueError(f"k shape {tuple(k.shape)} does not match the cache (B={c.B}, H={c.H}, d={c.d})")
+        _need(v, torch.bfloat16, tuple(k.shape), "v")
+        _check(load().bsva_kv_cache_append(ctypes.byref(c), _ptr(k), _ptr(v), k.shape[2], _stream(stream)))
+
+    def workspace_bytes(self, Lq: int) -> int:
+        n = load().bsva_kv_cache_workspace_bytes(ctypes.byref(self.c), Lq)
+        if n == 0:
+            raise BsvaError(1, f"bad cache geometry or Lq = {Lq}")
+        return n
+
+    def attend(self, qq: dict, block_mask: torch.Tensor, softmax_scale: float = 0.0, with_lse: bool = False,
+               workspace=None, out=None, lse=None, out_dtype=torch.bfloat16, stream=None):
+        """The mask entry over the live slabs (C ABI ``masked_block_attn_fwd_kvcache``); ``qq`` from
+        ``quantize_q``, ``block_mask`` uint8 [B, Hm, nQB, count] over the live slabs, oldest first."""
+        c = self.c
+        q8, q_scale = qq["q8"], qq["q_scale"]
+        _need(q8, torch.int8, None, "q8")
+        if q8.dim() != 4 or tuple(q8.shape[:2]) != (c.B, c.H) or q8.shape[3] != c.d:
+            raise ValueError(f"q8 shape {tuple(q8.shape)} does not match the cache")
+        B, H, Lq, d = q8.shape
+        _need(block_mask, torch.uint8, None, "block_mask")
+        if block_mask.dim() != 4 or block_mask.shape[0] != B or tuple(block_mask.shape[2:]) != (-(-Lq // 128), c.count):
+            raise ValueError(f"block_mask shape {tuple(block_mask.shape)} is not [B, Hm, nQB, live slabs]")
+        if workspace is None:
+            workspace = torch.zeros(self.workspace_bytes(Lq), dtype=torch.uint8, device=q8.device)
+        out = _out(out, (B, H, Lq, d), out_dtype, q8.device)
+        if with_lse and lse is None:
+            lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q8.device)
+        _check(load().masked_block_attn_fwd_kvcache(ctypes.byref(c), Lq, _ptr(q8), _ptr(q_scale), _ptr(block_mask),
+                                                    block_mask.shape[1], ctypes.c_float(softmax_scale),
+                                                    OUT_DTYPES[out.dtype], _ptr(out), _ptr(lse), _ptr(workspace),
+                                                    workspace.numel(), _stream(stream)))
+        return (out, lse) if with_lse else out

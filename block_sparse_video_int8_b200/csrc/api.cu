@@ -131,20 +131,28 @@ int check_workspace(void* ws, size_t bytes, size_t need) {
 }
 
 // Shared tail of both attention entry points.
+// The INT8 streaming cache as the key side of an attention launch: the K/V maps cover all
+// ring slots, key block j lives in slot (first + j / 2) % slots.
+struct RingArgs {
+  const int32_t* slab_rows = nullptr;
+  int first = 0, slots = 0;
+};
+
 int run_attention(const bsva_shape& s, const int8_t* q8, const float* q_scale, const int8_t* k8,
                   const float* k_scale, const void* v, const uint8_t* kept_mask, const int32_t* kept_idx,
                   const int32_t* kept_cnt, int centroid_mode, float softmax_scale, int out_dtype, void* out,
                   float* lse, unsigned char* ws, const WsLayout& L, cudaStream_t st,
-                  const float* v_scale = nullptr, const int2* vtab = nullptr) {
+                  const float* v_scale = nullptr, const int2* vtab = nullptr, const RingArgs& ring = RingArgs()) {
   int rc = get_encoder();
   if (rc) return rc;
   const uint64_t BH = uint64_t(s.B) * s.H;
+  const uint64_t krows = ring.slab_rows ? uint64_t(ring.slots) * 128 : uint64_t(s.Lk);   // rows of the K/V maps
   AttnMaps maps;
   const CUtensorMapSwizzle swq = s.d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   if ((rc = encode_map(&maps.q8, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.d, s.Lq, BH, s.d, QB, swq, "q8"))) return rc;
-  if ((rc = encode_map(&maps.k8, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.d, s.Lk, BH, s.d, KB, swq, "k8"))) return rc;
+  if ((rc = encode_map(&maps.k8, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.d, krows, BH, s.d, KB, swq, "k8"))) return rc;
   if (v_scale) {   // INT8 V: whole rows of d bytes, widened in shared memory by the kernel
-    if ((rc = encode_map(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.d, s.Lk, BH, s.d, KB,
+    if ((rc = encode_map(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, s.d, krows, BH, s.d, KB,
                          CU_TENSOR_MAP_SWIZZLE_NONE, "v8")))
       return rc;
   } else if ((rc = encode_map(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, s.d, s.Lk, BH, 64, KB,
@@ -180,6 +188,9 @@ int run_attention(const bsva_shape& s, const int8_t* q8, const float* q_scale, c
   a.cbias = centroid_mode > 0 ? reinterpret_cast<const float*>(ws + L.cbias) : nullptr;
   a.vtab = vtab;
   a.n_vtiles = vtab ? L.n_vtiles : 0;
+  a.slab_rows = ring.slab_rows;
+  a.ring_first = ring.first;
+  a.ring_slots = ring.slots;
   a.out = out_dtype == BSVA_OUT_BF16 ? reinterpret_cast<__nv_bfloat16*>(out) : nullptr;
   a.out_f32 = out_dtype == BSVA_OUT_F32 ? reinterpret_cast<float*>(out) : nullptr;
   a.lse = lse;
@@ -461,6 +472,107 @@ int masked_block_attn_fwd_v8(bsva_shape s, const int8_t* q8, const float* q_scal
   if (e != cudaSuccess) return cuda_fail(e, "mask expansion launch");
   return run_attention(s, q8, q_scale, k8, k_scale, v8, nullptr, kidx, kcnt, 0, softmax_scale, out_dtype, out, lse,
                        ws, L, st, v_scale);
+}
+
+int bsva_quantize_q(bsva_shape s, const void* q, int8_t* q8, float* q_scale, int32_t* q_pool, bsva_stream_t stream) {
+  BSVA_RANGE("bsva_quantize_q");
+  int rc;
+  s.Lk = s.Lq;   // not used; keeps the shape check meaningful
+  if ((rc = check_shape(s))) return rc;
+  REQUIRE_PTR(q, 16); REQUIRE_PTR(q8, 16); REQUIRE_PTR(q_scale, 4); REQUIRE_PTR(q_pool, 16);
+  if ((rc = check_device())) return rc;
+  cudaError_t e = launch_quant_q(s, reinterpret_cast<const __nv_bfloat16*>(q), q8, q_scale, q_pool,
+                                 reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "Q quantiser launch");
+  return ok();
+}
+
+static int check_kv_cache(const bsva_kv_cache* c) {
+  if (c == nullptr) return fail(BSVA_ERR_INVALID_ARG, "cache is NULL");
+  if (c->B < 1 || c->H < 1 || size_t(c->B) * c->H > 65535u)
+    return fail(BSVA_ERR_INVALID_ARG, "cache: B, H must be >= 1 with B*H <= 65535 (got %d, %d)", c->B, c->H);
+  if (c->d != 64 && c->d != 128) return fail(BSVA_ERR_UNSUPPORTED, "cache head dim d = %d; supported: 64, 128", c->d);
+  if (c->n_slots < 1 || c->n_slots > (1 << 22)) return fail(BSVA_ERR_INVALID_ARG, "cache n_slots = %d", c->n_slots);
+  if (c->first < 0 || c->first >= c->n_slots || c->count < 0 || c->count > c->n_slots)
+    return fail(BSVA_ERR_INVALID_ARG, "cache ring state first = %d, count = %d outside [0, %d)", c->first, c->count,
+                c->n_slots);
+  REQUIRE_PTR(c->k8, 16); REQUIRE_PTR(c->v8, 16); REQUIRE_PTR(c->k_scale, 4); REQUIRE_PTR(c->v_scale, 4);
+  REQUIRE_PTR(c->slab_rows, 4);
+  return BSVA_OK;
+}
+
+int bsva_kv_cache_append(bsva_kv_cache* c, const void* k, const void* v, int Lc, bsva_stream_t stream) {
+  BSVA_RANGE("bsva_kv_cache_append");
+  int rc;
+  if ((rc = check_kv_cache(c))) return rc;
+  if (Lc < 1 || Lc > (1 << 30)) return fail(BSVA_ERR_INVALID_ARG, "chunk length %d", Lc);
+  REQUIRE_PTR(k, 16); REQUIRE_PTR(v, 16);
+  if ((rc = check_device())) return rc;
+  const int nslabs = (Lc + 127) / 128;
+  const int skip = nslabs > c->n_slots ? nslabs - c->n_slots : 0;   // leading slabs that would be evicted at once
+  const int kept = nslabs - skip;
+  // evict the oldest slabs to make room, then the chunk's slabs follow the newest one
+  const int evict = c->count + kept > c->n_slots ? c->count + kept - c->n_slots : 0;
+  const int first = (c->first + evict) % c->n_slots;
+  const int count = c->count - evict;
+  const int slot0 = (first + count) % c->n_slots;
+  cudaError_t e = launch_kv_append(*c, reinterpret_cast<const __nv_bfloat16*>(k),
+                                   reinterpret_cast<const __nv_bfloat16*>(v), Lc, skip, slot0,
+                                   reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cache append launch");
+  c->first = count + kept > 0 ? first : 0;
+  c->count = count + kept;
+  return ok();
+}
+
+static bsva_shape kv_cache_shape(const bsva_kv_cache* c, int Lq) {
+  bsva_shape s{};
+  s.B = c->B; s.H = c->H; s.Lq = Lq; s.Lk = 128 * (c->count > 0 ? c->count : 1); s.d = c->d; s.n_prefix = 0;
+  return s;
+}
+
+size_t bsva_kv_cache_workspace_bytes(const bsva_kv_cache* c, int Lq) {
+  if (check_kv_cache(c) != BSVA_OK || Lq < 1) return 0;
+  const bsva_shape s = kv_cache_shape(c, Lq);
+  if (check_shape(s) != BSVA_OK) return 0;
+  return ws_layout(s, 0).total;
+}
+
+int masked_block_attn_fwd_kvcache(const bsva_kv_cache* c, int Lq, const int8_t* q8, const float* q_scale,
+                                  const uint8_t* block_mask, int mask_heads, float softmax_scale, int out_dtype,
+                                  void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                  bsva_stream_t stream) {
+  BSVA_RANGE("masked_block_attn_fwd_kvcache");
+  int rc;
+  if ((rc = check_kv_cache(c))) return rc;
+  if (c->count < 1) return fail(BSVA_ERR_INVALID_ARG, "the cache holds no slab");
+  if (Lq < 1) return fail(BSVA_ERR_INVALID_ARG, "Lq = %d", Lq);
+  const bsva_shape s = kv_cache_shape(c, Lq);
+  if ((rc = check_shape(s))) return rc;
+  if (mask_heads != 1 && mask_heads != s.H)
+    return fail(BSVA_ERR_INVALID_ARG, "mask_heads = %d must be 1 or H = %d", mask_heads, s.H);
+  if (std::isnan(softmax_scale) || std::isinf(softmax_scale))
+    return fail(BSVA_ERR_INVALID_ARG, "softmax_scale must be finite");
+  if (out_dtype != BSVA_OUT_BF16 && out_dtype != BSVA_OUT_F32)
+    return fail(BSVA_ERR_INVALID_ARG, "out_dtype = %d; use BSVA_OUT_BF16 (0) or BSVA_OUT_F32 (1)", out_dtype);
+  REQUIRE_PTR(q8, 16); REQUIRE_PTR(q_scale, 4); REQUIRE_PTR(block_mask, 1); REQUIRE_PTR(out, 16);
+  if (lse && !aligned(lse, 4)) return fail(BSVA_ERR_INVALID_ARG, "lse is not 4-byte aligned");
+  const WsLayout L = ws_layout(s, 0);
+  if ((rc = check_workspace(workspace, workspace_bytes, L.total))) return rc;
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  int32_t* kidx = reinterpret_cast<int32_t*>(ws + L.kidx);
+  int32_t* kcnt = reinterpret_cast<int32_t*>(ws + L.kcnt);
+  const int nQB = (Lq + QB - 1) / QB;
+  cudaError_t e = launch_kv_mask_expand(*c, nQB, block_mask, mask_heads, kidx, kcnt, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cache mask expansion launch");
+  RingArgs ring;
+  ring.slab_rows = c->slab_rows;
+  ring.first = c->first;
+  ring.slots = c->n_slots;
+  return run_attention(s, q8, q_scale, c->k8, c->k_scale, c->v8, nullptr, kidx, kcnt, 0, softmax_scale, out_dtype,
+                       out, lse, ws, L, st, c->v_scale, nullptr, ring);
 }
 
 static int check_virtual_geometry(int slice_tokens, int n_src_slices, int centroid_mode) {

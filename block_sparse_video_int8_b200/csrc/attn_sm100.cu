@@ -32,6 +32,9 @@
 // f16; the block scale s_j is folded into the exponent, P' = 2^(y + log2 s_j),
 // and the row sums take the rounded P' times 2^-log2 s_j, so numerator and
 // denominator weight each key alike.
+// The same instantiation reads the INT8 streaming cache: key block j of the
+// cache is 64-row block j mod 2 of the slab in ring slot (first + j / 2) mod
+// n_slots (a.slab_rows non-null).
 // Centroid tiles hold 32 groups as (hi, lo) INT8 row pairs (pool = 128 hi + lo)
 // so their dot with q8 is exact in int32; the value rows are (bf16 hi, bf16 lo)
 // and share one probability.
@@ -95,6 +98,13 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Physical 64-row block of logical key block j: itself, or in the INT8 streaming cache the
+// block of the slab in ring slot (first + j / 2) mod n_slots.
+__device__ __forceinline__ int phys_block(const AttnArgs& a, int j) {
+  if (a.slab_rows == nullptr) return j;
+  return ((a.ring_first + (j >> 1)) % a.ring_slots) * 2 + (j & 1);
 }
 
 // kV8: V is INT8 with per-block scales (a.v_scale), P and V enter PV as f16.
@@ -168,6 +178,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // their scales are fetched 32 tiles at a time, one per lane; centroid
     // metadata is fetched a tile ahead, one group per lane. Lane 0 issues TMA.
     const float sqs = a.q_scale[row_item] * a.scale_log2e;
+    const int scale_stride = a.slab_rows ? 2 * a.ring_slots : a.nKB;   // per-head count of K/V block scales
     const int32_t* kidx = a.kept_idx + row_item * a.nKB;
     const uint8_t* kmask = a.kept_mask ? a.kept_mask + row_item * a.nKB : nullptr;
     const float* cfac = a.cfac ? a.cfac + size_t(bh) * a.nCT * 32 : nullptr;
@@ -213,18 +224,18 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (t < n_exact) {
         if ((t & 31) == 0) {
           const int nn = t + lane;
-          chunk_j = nn < n_exact ? kidx[nn] : 0;
-          chunk_f = nn < n_exact ? sqs * a.k_scale[size_t(bh) * a.nKB + chunk_j] : 0.f;
+          chunk_j = nn < n_exact ? phys_block(a, kidx[nn]) : 0;
+          chunk_f = nn < n_exact ? sqs * a.k_scale[size_t(bh) * scale_stride + chunk_j] : 0.f;
         }
         j_next = __shfl_sync(0xffffffffu, chunk_j, t & 31);
         const float f_next = __shfl_sync(0xffffffffu, chunk_f, t & 31);
         row = j_next * KB;
         if (lane == 0) {
           mt.f = f_next;
-          mt.nvalid = min(KB, a.Lk - row);
+          mt.nvalid = a.slab_rows ? min(KB, a.slab_rows[j_next >> 1] - (j_next & 1) * KB) : min(KB, a.Lk - row);
           mt.centroid = 0;
           if constexpr (kV8) {
-            const float sv = a.v_scale[size_t(bh) * a.nKB + j_next];
+            const float sv = a.v_scale[size_t(bh) * scale_stride + j_next];
             mt.vlog2 = sv > 0.f ? __log2f(sv) : 0.f;
           }
         }

@@ -334,6 +334,9 @@ struct AttnArgs {
   const float* cfac;        // [BH, nCT*32]
   const float* cbias;       // [BH, nCT*32]
   const int2* vtab;         // virtual K/V: [n_vtiles] (first source group, live groups); null otherwise
+  const int32_t* slab_rows; // INT8 streaming cache: [ring_slots] valid rows per slot; null otherwise
+  int ring_first;           // cache: ring slot of the oldest live slab
+  int ring_slots;           // cache: slots in the ring
   int n_vtiles;             // virtual K/V: centroid tiles of every query block
   __nv_bfloat16* out;       // [BH, Lq, d] bf16 output, or
   float* out_f32;           // [BH, Lq, d] fp32 output (exactly one is non-null)
@@ -349,6 +352,9 @@ struct AttnMaps {
 cudaError_t launch_quant_pool(const bsva_shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, int8_t* q8,
                               float* q_scale, int8_t* k8, float* k_scale, int32_t* q_pool, int32_t* k_pool,
                               cudaStream_t st);
+// The Q half alone (query codes, scales and pools).
+cudaError_t launch_quant_q(const bsva_shape& s, const __nv_bfloat16* q, int8_t* q8, float* q_scale, int32_t* q_pool,
+                           cudaStream_t st);
 // The K quantiser alone over another [B, H, Lk, d] tensor (INT8 V), no pools.
 cudaError_t launch_quant_v(const bsva_shape& s, const __nv_bfloat16* v, int8_t* v8, float* v_scale, cudaStream_t st);
 cudaError_t launch_route(const bsva_shape& s, double tau, const int32_t* q_pool, const int32_t* k_pool,
@@ -370,6 +376,12 @@ cudaError_t launch_dense_lists(const bsva_shape& s, int32_t* kept_idx, int32_t* 
 cudaError_t launch_virtual_tiles(const int* src_map, int n_virtual, int groups_per_slice, int2* vtab,
                                  cudaStream_t st);
 cudaError_t launch_attention(const AttnArgs& a, const AttnMaps& maps, cudaStream_t st);
+// INT8 streaming cache: quantise a chunk into its slabs (slot0 = slot of the first written
+// slab, skip_slabs leading slabs of the chunk dropped), and the kept lists over the live slabs.
+cudaError_t launch_kv_append(const bsva_kv_cache& c, const __nv_bfloat16* k, const __nv_bfloat16* v, int Lc,
+                             int skip_slabs, int slot0, cudaStream_t st);
+cudaError_t launch_kv_mask_expand(const bsva_kv_cache& c, int nQB, const uint8_t* block_mask, int mask_heads,
+                                  int32_t* kept_idx, int32_t* kept_cnt, cudaStream_t st);
 cudaError_t launch_selftest_timeout(uint32_t* status, uint64_t limit_ns, cudaStream_t st);
 
 }  // namespace bsva

@@ -206,6 +206,18 @@ cudaError_t launch_quant_pool(const bsva_shape& s, const __nv_bfloat16* q, const
   return cudaGetLastError();
 }
 
+cudaError_t launch_quant_q(const bsva_shape& s, const __nv_bfloat16* q, int8_t* q8, float* q_scale, int32_t* q_pool,
+                           cudaStream_t st) {
+  dim3 grid((s.Lq + QB - 1) / QB, s.B * s.H, 1);
+  if (s.d == 128)
+    quant_pool_kernel<128><<<grid, kThreads, 0, st>>>(q, nullptr, q8, q_scale, nullptr, nullptr, q_pool, nullptr,
+                                                      s.Lq, s.Lk, 0);
+  else
+    quant_pool_kernel<64><<<grid, kThreads, 0, st>>>(q, nullptr, q8, q_scale, nullptr, nullptr, q_pool, nullptr,
+                                                     s.Lq, s.Lk, 0);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quant_v(const bsva_shape& s, const __nv_bfloat16* v, int8_t* v8, float* v_scale, cudaStream_t st) {
   dim3 grid((s.Lk + QB - 1) / QB, s.B * s.H, 1);
   if (s.d == 128)

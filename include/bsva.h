@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define BSVA_ABI_VERSION 3
+#define BSVA_ABI_VERSION 4
 
 enum bsva_status {
   BSVA_OK = 0,
@@ -300,6 +300,71 @@ int virtual_kv_residual_fwd(bsva_shape s, const int8_t* q8, const float* q_scale
                             int centroid_mode, float softmax_scale, int out_dtype,
                             void* out, float* lse, void* workspace,
                             size_t workspace_bytes, bsva_stream_t stream);
+
+/* Per-block INT8 quantisation of Q alone (128-row blocks, the quantiser of
+ * bsva_quantize_qk), for queries that attend to keys quantised elsewhere,
+ * such as the INT8 streaming cache below. s.Lk is not used.
+ *   q        bf16 [B,H,Lq,d]
+ *   q8       out: int8 [B,H,Lq,d];  q_scale out: fp32 [B,H,nQB]
+ *   q_pool   out: int32 [B,H,nQB,d] (column sums of each block's codes)         */
+int bsva_quantize_q(bsva_shape s, const void* q, int8_t* q8, float* q_scale,
+                    int32_t* q_pool, bsva_stream_t stream);
+
+/* INT8 streaming K/V cache in 128-row slabs ("FlashVSR Kitchen Sparse
+ * Attention", intro: the streaming modes keep a sliding cache of past K and V
+ * as INT8 and hand bounded 128-row slabs straight to the sparse kernel, with
+ * no full-precision rebuild; When it bites: the INT8 path needs an INT8 cache
+ * to feed). Per (batch, head) the cache is a ring of n_slots slabs: logical
+ * slab x (0 = the oldest live slab) sits in slot (first + x) % n_slots. A slab
+ * holds up to 128 consecutive tokens of one appended chunk; its K and V are
+ * quantised in 64-row blocks with the K quantiser (s = fl32(amax/127), codes
+ * rint_half_even(fl32(x/s)) over the block's valid rows).
+ * The caller allocates the device buffers (zero-initialised or not: nothing is
+ * read before it is written) and owns the struct; bsva_kv_cache_append updates
+ * first and count. Start with first = count = 0. */
+typedef struct bsva_kv_cache {
+  int B, H, d;          /* heads and head dim of every chunk (d = 64 or 128)      */
+  int n_slots;          /* capacity in slabs, >= 1                                */
+  int8_t* k8;           /* device int8 [B, H, n_slots*128, d]                     */
+  float* k_scale;       /* device fp32 [B, H, n_slots*2], one per 64-row block    */
+  int8_t* v8;           /* device int8 [B, H, n_slots*128, d]                     */
+  float* v_scale;       /* device fp32 [B, H, n_slots*2]                          */
+  int32_t* slab_rows;   /* device int32 [n_slots]: valid rows of each slot's slab */
+  int first;            /* slot of the oldest live slab                           */
+  int count;            /* live slabs                                             */
+} bsva_kv_cache;
+
+/* Appends a chunk of Lc >= 1 new tokens, k and v bf16 [B, H, Lc, d]. The chunk
+ * becomes ceil(Lc/128) slabs, the last one holding Lc - 128*(ceil(Lc/128)-1)
+ * rows. When the ring would overflow, the oldest slabs are evicted first; a
+ * chunk longer than the whole ring keeps only its last n_slots slabs.
+ * c->first and c->count are updated on the host when the call returns; the
+ * quantisation runs on `stream`. Returns BSVA_ERR_INVALID_ARG for a bad
+ * geometry or pointer, leaving the cache untouched. */
+int bsva_kv_cache_append(bsva_kv_cache* c, const void* k, const void* v, int Lc,
+                         bsva_stream_t stream);
+
+/* Workspace bytes of masked_block_attn_fwd_kvcache for Lq query tokens against
+ * the cache's current live slabs; 0 on a bad geometry. */
+size_t bsva_kv_cache_workspace_bytes(const bsva_kv_cache* c, int Lq);
+
+/* The mask entry over the live slabs of the INT8 cache, reading INT8 K and V
+ * straight from their slots (no copy, no bf16 rebuild). The keys are the valid
+ * rows of the live slabs, oldest first; one logical mask column per live slab
+ * (a slab is a 128-key logical block). The output is softmax attention over
+ * the dequantised cache, exact terms only, as in masked_block_attn_fwd_v8.
+ *   Lq            query tokens
+ *   q8, q_scale   int8 [B,H,Lq,d], fp32 [B,H,nQB] (bsva_quantize_q)
+ *   block_mask    uint8 [B, mask_heads, nQB, c->count]: query block i attends
+ *                 to logical slab x iff block_mask[b, h % mask_heads, i, x] != 0
+ *   workspace     >= bsva_kv_cache_workspace_bytes(c, Lq) bytes, 256-aligned
+ *   Other arguments as in masked_block_attn_fwd. A query row with no allowed
+ *   key gets out = 0 and lse = -inf. */
+int masked_block_attn_fwd_kvcache(const bsva_kv_cache* c, int Lq, const int8_t* q8,
+                                  const float* q_scale, const uint8_t* block_mask,
+                                  int mask_heads, float softmax_scale, int out_dtype,
+                                  void* out, float* lse, void* workspace,
+                                  size_t workspace_bytes, bsva_stream_t stream);
 
 /* masked_block_attn_fwd without a workspace. The source pages have no
  * counterpart: this entry point is for callers that cannot allocate device

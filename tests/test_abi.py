@@ -32,7 +32,7 @@ def test_library_builds_and_exports_every_declared_symbol():
 
 
 def test_abi_version_matches_binding():
-    assert bsva.abi_version() == bsva.ABI_VERSION == 3
+    assert bsva.abi_version() == bsva.ABI_VERSION == 4
 
 
 def test_workspace_size_arithmetic():
@@ -200,3 +200,45 @@ def test_virtual_kv_binding_refuses_cpu_tensors():
     v = torch.zeros((1, 1, 640, 128), dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         bsva.virtual_kv_residual_fwd(qk, v, 320, (0, 1))
+
+
+def _cache(n_slots=4, d=128, B=1, H=2, first=0, count=0, ptr=0x10000):
+    P = ptr
+    return bsva.KVCacheStruct(B, H, d, n_slots, P, P, P, P, P, first, count)
+
+
+def test_kv_cache_entries_reject_bad_arguments():
+    lib = bsva.load()
+    P = ctypes.c_void_p(0x10000)
+    c = _cache()
+    assert lib.bsva_kv_cache_append(None, P, P, 128, None) == 1
+    assert lib.bsva_kv_cache_append(ctypes.byref(c), P, P, 0, None) == 1          # empty chunk
+    assert lib.bsva_kv_cache_append(ctypes.byref(c), None, P, 128, None) == 1
+    bad_d = _cache(d=96)
+    assert lib.bsva_kv_cache_append(ctypes.byref(bad_d), P, P, 128, None) == 2
+    bad_ring = _cache(first=4)                                                     # first outside [0, n_slots)
+    assert lib.bsva_kv_cache_append(ctypes.byref(bad_ring), P, P, 128, None) == 1
+    assert (bad_ring.first, bad_ring.count) == (4, 0)                              # untouched on failure
+    misaligned = _cache(ptr=0x10001)
+    assert lib.bsva_kv_cache_append(ctypes.byref(misaligned), P, P, 128, None) == 1
+    # the attention entry: an empty cache, a wrong mask head count, a small workspace
+    rc = lib.masked_block_attn_fwd_kvcache(ctypes.byref(c), 256, P, P, P, 1, ctypes.c_float(0), 0, P, None, P,
+                                           1 << 30, None)
+    assert rc == 1 and b"no slab" in lib.bsva_last_error()
+    live = _cache(count=3, first=2)
+    rc = lib.masked_block_attn_fwd_kvcache(ctypes.byref(live), 256, P, P, P, 3, ctypes.c_float(0), 0, P, None, P,
+                                           1 << 30, None)
+    assert rc == 1
+    rc = lib.masked_block_attn_fwd_kvcache(ctypes.byref(live), 256, P, P, P, 1, ctypes.c_float(0), 0, P, None, P,
+                                           64, None)
+    assert rc == 3
+    # workspace: kept lists over the live slabs' 64-row blocks, one row per query block
+    n = lib.bsva_kv_cache_workspace_bytes(ctypes.byref(live), 256)
+    assert n >= 1 * 2 * 2 * 6 * 4 and lib.bsva_kv_cache_workspace_bytes(ctypes.byref(live), 0) == 0
+    assert lib.bsva_quantize_q(bsva.Shape(1, 2, 256, 256, 128, 0), P, None, P, P, None) == 1
+
+
+def test_kv_cache_binding_refuses_cpu_tensors():
+    k = torch.zeros((1, 2, 128, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        bsva.quantize_q(k)
