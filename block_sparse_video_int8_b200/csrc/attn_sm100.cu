@@ -10,11 +10,14 @@
 //   warps 0-3  softmax: thread r owns query row r (TMEM lane r). Reads S from
 //              TMEM, scales, online max/sum, writes P (bf16) back to TMEM,
 //              rescales O in TMEM when the running max grows by more than
-//              2^8, and runs the epilogue O / l.
+//              2^8, and runs the epilogue O / l. The weights are computed
+//              against the running max first; the tile max is taken only
+//              when some row's weights sum to more than 2^8.
 //   warp 4     TMA producer: Q tile once, then K (int8) tiles with their
 //              per-tile metadata into a 4-stage ring (freed by the softmax
 //              warps once they are done with the tile), first the kept
-//              blocks, then the centroid tiles.
+//              blocks, starting at the query block's own keys and wrapping
+//              round, then the centroid tiles.
 //   warp 5     TMEM owner (alloc/dealloc) and MMA issuer (the warp runs the
 //              schedule, one elected lane issues); it also loads the V
 //              (bf16) tiles into a 3-stage ring, two tiles ahead of PV, as
@@ -190,6 +193,31 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_arrive_expect_tx(&sm.q_full, QB * D);
       tma_load_3d(sm.q, &maps.q8, 0, q0, bh, &sm.q_full);
     }
+    // The kept tiles run from the first kept block at or after the query block's own keys (the
+    // key block at the middle of its rows, the ends of the two sequences aligned), wrapping round:
+    // the largest logits of a row then come first, so the running max seldom has to grow later.
+    int rot = 0;
+    if (n_exact > 1) {
+      const int jstar = min(max((q0 + QB / 2 + a.Lk - a.Lq) / KB, 0), a.nKB - 1);
+      // count the kept indices below jstar (the list ascends): narrow with 32 probes per round
+      int lo = 0, len = n_exact;   // every index before lo is below jstar; the count is in [lo, lo + len]
+      while (len > 32) {
+        const int step = (len + 31) / 32;
+        const int x = lo + lane * step;
+        const bool below = x < lo + len && kidx[x] < jstar;
+        const int c = __popc(__ballot_sync(0xffffffffu, below));
+        if (c == 0) {
+          len = 0;
+        } else {
+          const int nlo = lo + (c - 1) * step + 1;
+          len = min(step - 1, lo + len - nlo);
+          lo = nlo;
+        }
+      }
+      const bool below = lane < len && kidx[lo + lane] < jstar;
+      rot = lo + __popc(__ballot_sync(0xffffffffu, below));
+      if (rot >= n_exact) rot = n_exact - 1;
+    }
     int chunk_j = 0;          // kept index of tile (32*c + lane) of the current chunk
     float chunk_f = 0.f;
     int j_next = 0;              // key block of the K step's tile
@@ -224,7 +252,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (t < n_exact) {
         if ((t & 31) == 0) {
           const int nn = t + lane;
-          chunk_j = nn < n_exact ? phys_block(a, kidx[nn]) : 0;
+          const int pos = nn + rot < n_exact ? nn + rot : nn + rot - n_exact;
+          chunk_j = nn < n_exact ? phys_block(a, kidx[pos]) : 0;
           chunk_f = nn < n_exact ? sqs * a.k_scale[size_t(bh) * scale_stride + chunk_j] : 0.f;
         }
         j_next = __shfl_sync(0xffffffffu, chunk_j, t & 31);
@@ -508,30 +537,38 @@ __global__ void __launch_bounds__(kThreads, 2)
         };
         // Speculate that the running max still holds (it nearly always does
         // after the first tiles), so the exps need not wait for this tile's max.
+        // The tile max is needed only where some weight may exceed 2^8 (a logit
+        // above m_ref + 8): a row whose weights sum to at most 2^8 has none.
         const bool first = __all_sync(0xffffffffu, m_ref == -INFINITY);
-        if (!first) exps(m_ref);
-        float m8[22];
+        bool check = first;
+        if (!first) {
+          exps(m_ref);
+          check = __any_sync(0xffffffffu, !(lsum <= 256.f));
+        }
+        if (check) {
+          float m8[22];
 #pragma unroll
-        for (int c = 0; c < 21; ++c) m8[c] = fmax3(xs[3 * c], xs[3 * c + 1], xs[3 * c + 2]);
-        m8[21] = xs[63];
+          for (int c = 0; c < 21; ++c) m8[c] = fmax3(xs[3 * c], xs[3 * c + 1], xs[3 * c + 2]);
+          m8[21] = xs[63];
 #pragma unroll
-        for (int c = 0; c < 7; ++c) m8[c] = fmax3(m8[3 * c], m8[3 * c + 1], m8[3 * c + 2]);
-        m8[0] = fmax3(m8[0], m8[1], m8[2]);
-        m8[1] = fmax3(m8[3], m8[4], m8[5]);
-        m8[2] = fmax3(m8[6], m8[21], m8[0]);
-        const float mt_max = fmaxf(m8[1], m8[2]) * f;   // f > 0: the max commutes with the scale
-        const bool need = mt_max > m_ref + kRescaleLog2;
-        if (first || __any_sync(0xffffffffu, need)) {
-          const float m_new = need ? mt_max : m_ref;
-          const float alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new);
-          if (n > 0 && !rescale_o(alpha)) {
-            alive = false;
-            break;
+          for (int c = 0; c < 7; ++c) m8[c] = fmax3(m8[3 * c], m8[3 * c + 1], m8[3 * c + 2]);
+          m8[0] = fmax3(m8[0], m8[1], m8[2]);
+          m8[1] = fmax3(m8[3], m8[4], m8[5]);
+          m8[2] = fmax3(m8[6], m8[21], m8[0]);
+          const float mt_max = fmaxf(m8[1], m8[2]) * f;   // f > 0: the max commutes with the scale
+          const bool need = mt_max > m_ref + kRescaleLog2;
+          if (first || __any_sync(0xffffffffu, need)) {
+            const float m_new = need ? mt_max : m_ref;
+            const float alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new);
+            if (n > 0 && !rescale_o(alpha)) {
+              alive = false;
+              break;
+            }
+            l *= alpha;
+            le *= alpha;
+            m_ref = m_new;
+            exps(m_ref == -INFINITY ? 0.f : m_ref);
           }
-          l *= alpha;
-          le *= alpha;
-          m_ref = m_new;
-          exps(m_ref == -INFINITY ? 0.f : m_ref);
         }
       } else {
         // ---- centroid tile: 32 groups, each an exact int dot from its (hi, lo) rows
@@ -551,32 +588,49 @@ __global__ void __launch_bounds__(kThreads, 2)
           const int dot = 128 * int(sb[2 * g]) + int(sb[2 * g + 1]);
           xs[16 + g] = fmaf(float(dot), mt.fac[16 + g], mt.bias[16 + g]);
         }
-        float m8[11];
+        auto cexps = [&](float m_use) {
+          float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-        for (int c = 0; c < 10; ++c) m8[c] = fmax3(xs[3 * c], xs[3 * c + 1], xs[3 * c + 2]);
-        m8[10] = fmaxf(xs[30], xs[31]);
-        m8[0] = fmax3(m8[0], m8[1], m8[2]);
-        m8[1] = fmax3(m8[3], m8[4], m8[5]);
-        m8[2] = fmax3(m8[6], m8[7], m8[8]);
-        const float mt_max = fmax3(fmax3(m8[0], m8[1], m8[2]), m8[9], m8[10]);
-        const bool need = mt_max > m_ref + kRescaleLog2;
-        if (__any_sync(0xffffffffu, need)) {
-          const float m_new = need ? mt_max : m_ref;
-          const float alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new);
-          if (n > 0 && !rescale_o(alpha)) {
-            alive = false;
-            break;
+          for (int g = 0; g < 32; g += 2) {
+            const float p0 = ex2(xs[g] - m_use), p1 = ex2(xs[g + 1] - m_use);
+            pk[g] = pack_bf16x2(p0, p0);
+            pk[g + 1] = pack_bf16x2(p1, p1);
+            s0 += p0;
+            s1 += p1;
           }
-          l *= alpha;
-          le *= alpha;
-          m_ref = m_new;
+          lsum = s0 + s1;
+        };
+        // as for kept tiles: speculate on the running max, take the tile max only where the
+        // weights of some row sum to more than 2^8
+        const bool first = __all_sync(0xffffffffu, m_ref == -INFINITY);
+        bool check = first;
+        if (!first) {
+          cexps(m_ref);
+          check = __any_sync(0xffffffffu, !(lsum <= 256.f));
         }
-        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        if (check) {
+          float m8[11];
 #pragma unroll
-        for (int g = 0; g < 32; ++g) {
-          const float p = ex2(xs[g] - m_use);
-          pk[g] = pack_bf16x2(p, p);
-          lsum += p;
+          for (int c = 0; c < 10; ++c) m8[c] = fmax3(xs[3 * c], xs[3 * c + 1], xs[3 * c + 2]);
+          m8[10] = fmaxf(xs[30], xs[31]);
+          m8[0] = fmax3(m8[0], m8[1], m8[2]);
+          m8[1] = fmax3(m8[3], m8[4], m8[5]);
+          m8[2] = fmax3(m8[6], m8[7], m8[8]);
+          const float mt_max = fmax3(fmax3(m8[0], m8[1], m8[2]), m8[9], m8[10]);
+          const bool need = mt_max > m_ref + kRescaleLog2;
+          const bool any_need = __any_sync(0xffffffffu, need);
+          if (any_need) {
+            const float m_new = need ? mt_max : m_ref;
+            const float alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new);
+            if (n > 0 && !rescale_o(alpha)) {
+              alive = false;
+              break;
+            }
+            l *= alpha;
+            le *= alpha;
+            m_ref = m_new;
+          }
+          if (first || any_need) cexps(m_ref == -INFINITY ? 0.f : m_ref);
         }
         esum = lsum;
       }
