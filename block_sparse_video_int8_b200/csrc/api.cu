@@ -54,7 +54,6 @@ struct NvtxRange {
 };
 #define BSVA_RANGE(name) NvtxRange bsva_nvtx_range_(name)
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per device-side wait
 
 // ------------------------------------------------------------- device check
 int check_device() {
@@ -256,7 +255,8 @@ int sparse_attn_route(bsva_shape s, const void* q, const void* k, double tau, in
                                     reinterpret_cast<const __nv_bfloat16*>(k), q8, q_scale, k8, k_scale, q_pool,
                                     k_pool, st);
   if (e != cudaSuccess) return cuda_fail(e, "quant_pool launch");
-  e = launch_route(s, tau, q_pool, k_pool, k_scale, scores, kept_mask, kept_idx, kept_cnt, row_stats, st);
+  uint32_t* status = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(workspace) + ws.status);
+  e = launch_route(s, tau, q_pool, k_pool, k_scale, scores, kept_mask, kept_idx, kept_cnt, row_stats, status, st);
   if (e != cudaSuccess) return cuda_fail(e, "route launch");
   return ok();
 }
@@ -286,7 +286,9 @@ int sparse_attn_route_topk(bsva_shape s, const void* q, const void* k, double sp
                                     reinterpret_cast<const __nv_bfloat16*>(k), q8, q_scale, k8, k_scale, q_pool,
                                     k_pool, st);
   if (e != cudaSuccess) return cuda_fail(e, "quant_pool launch");
-  e = launch_route_topk(s, k_keep, q_pool, k_pool, k_scale, scores, kept_mask, kept_idx, kept_cnt, row_stats, st);
+  uint32_t* status = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(workspace) + ws.status);
+  e = launch_route_topk(s, k_keep, q_pool, k_pool, k_scale, scores, kept_mask, kept_idx, kept_cnt, row_stats, status,
+                        st);
   if (e != cudaSuccess) return cuda_fail(e, "top-k route launch");
   return ok();
 }

@@ -319,6 +319,8 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // Defined next to their kernels; called by api.cu after validation.
 namespace bsva {
 
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per device-side wait
+
 struct AttnArgs {
   int B, H, Lq, Lk, d, n_prefix;
   int nQB, nKB;
@@ -357,12 +359,13 @@ cudaError_t launch_quant_q(const bsva_shape& s, const __nv_bfloat16* q, int8_t* 
                            cudaStream_t st);
 // The K quantiser alone over another [B, H, Lk, d] tensor (INT8 V), no pools.
 cudaError_t launch_quant_v(const bsva_shape& s, const __nv_bfloat16* v, int8_t* v8, float* v_scale, cudaStream_t st);
+// status: the workspace status word (a score-kernel wait that runs out is recorded there).
 cudaError_t launch_route(const bsva_shape& s, double tau, const int32_t* q_pool, const int32_t* k_pool,
                          const float* k_scale, double* scores, uint8_t* kept_mask, int32_t* kept_idx,
-                         int32_t* kept_cnt, double* row_stats, cudaStream_t st);
+                         int32_t* kept_cnt, double* row_stats, uint32_t* status, cudaStream_t st);
 cudaError_t launch_route_topk(const bsva_shape& s, int k_keep, const int32_t* q_pool, const int32_t* k_pool,
                               const float* k_scale, double* scores, uint8_t* kept_mask, int32_t* kept_idx,
-                              int32_t* kept_cnt, double* row_stats, cudaStream_t st);
+                              int32_t* kept_cnt, double* row_stats, uint32_t* status, cudaStream_t st);
 cudaError_t launch_centroids(const bsva_shape& s, int centroid_mode, int nCT, const int32_t* k_pool,
                              const float* k_scale, const __nv_bfloat16* v, int8_t* ck8, __nv_bfloat16* cv,
                              float* cfac, float* cbias, cudaStream_t st);

@@ -34,79 +34,197 @@ namespace bsva {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kTile = 64;
+
+// ------------------------------------------------------------ proxy scores
+// Exact dots on the tensor core. Every pool value is split into two signed bytes,
+// x = 128 hi + lo with hi = floor((x + 64) / 128) and lo in [-64, 63]: |q_pool| <= 16256 and
+// |k_pool| <= 8128 keep hi in [-127, 127]. Then
+//   q . k = 16384 (qh . kh) + 128 (qh . kl + ql . kh) + (ql . kl),
+// three INT8 GEMMs with int32 accumulators (each below 127 * 127 * 2 * d < 2^23) combined in
+// int64. A CTA owns a tile of 128 query blocks x 64 key blocks: its four byte tiles go to shared
+// memory in the K-major swizzled layout tcgen05 reads (128-byte rows with the 128-byte swizzle
+// for d = 128, 64-byte rows with the 64-byte swizzle for d = 64), one thread issues the MMAs into
+// three 64-column TMEM accumulators, and each warp turns 32 rows x 32 key blocks of dots into
+// fp64 scores, fl(fl(dot * sk_j) / n_j) (n_j = 64 is a power of two, so the quotient is the
+// product with 1/64, bit for bit), staged through shared memory so that the stores run along
+// rows.
+constexpr int kSQ = 128;                   // query blocks per CTA (MMA M)
+constexpr int kSK = 64;                    // key blocks per CTA (MMA N)
+constexpr uint32_t kScoreTmemCols = 256;   // 3 x 64 used; two CTAs per SM
+constexpr int kStageLd = 17;               // doubles per staged row (16 + 1 against bank conflicts)
+
+template <int D>
+struct __align__(1024) ScoreSmem {
+  // the byte tiles; after the MMAs, the same bytes stage each warp's scores
+  union {
+    struct {
+      int8_t qh[kSQ * D];
+      int8_t ql[kSQ * D];
+      int8_t kh[kSK * D];
+      int8_t kl[kSK * D];
+    } t;
+    double stage[kThreads / 32][32 * kStageLd];
+  } u;
+  uint64_t done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Byte offset of (row r, byte c) of a K-major tile of D-byte rows in the swizzled layout: 8-row
+// atoms, the 16-byte chunk index XORed with address bits 7.. (row within the 1024-byte atom for
+// 128-byte rows, row / 2 within the 512-byte atom for 64-byte rows).
+template <int D>
+__device__ __forceinline__ uint32_t swz_offset(int r, int c) {
+  if (D == 128) return uint32_t((r >> 3) * 1024 + (r & 7) * 128 + ((((c >> 4) ^ (r & 7)) & 7) << 4) + (c & 15));
+  return uint32_t((r >> 3) * 512 + (r & 7) * 64 + ((((c >> 4) ^ ((r >> 1) & 3)) & 3) << 4) + (c & 15));
+}
+
+__device__ __forceinline__ void split_bytes(int4 x, uint32_t& hi, uint32_t& lo) {
+  const int v[4] = {x.x, x.y, x.z, x.w};
+  hi = 0;
+  lo = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int h = (v[e] + 64) >> 7;   // arithmetic shift: floor
+    const int l = v[e] - (h << 7);
+    hi |= uint32_t(h & 0xFF) << (8 * e);
+    lo |= uint32_t(l & 0xFF) << (8 * e);
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2) score_kernel(const int32_t* __restrict__ q_pool,
                                                             const int32_t* __restrict__ k_pool,
                                                             const float* __restrict__ k_scale,
-                                                            double* __restrict__ scores, int Lk, int nQB,
-                                                            int nKB) {
-  constexpr int KS = D + 4;
+                                                            double* __restrict__ scores, int Lk, int nQB, int nKB,
+                                                            uint32_t* status, uint64_t wait_limit_ns) {
+  extern __shared__ unsigned char smem_raw[];
+  ScoreSmem<D>& sm =
+      *reinterpret_cast<ScoreSmem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int bh = blockIdx.z, i0 = blockIdx.y * kSQ, j0 = blockIdx.x * kSK;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  if (t == 0) {
+    mbar_init(&sm.done, 1);
+    sm.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&sm.tmem_base, kScoreTmemCols);
+    tmem_relinquish();
+  }
+  // the byte tiles, four pool values (16 bytes in, 4 bytes out per tile) per step, 8 steps of
+  // loads in flight per thread
   constexpr int C4 = D / 4;
-  extern __shared__ __align__(16) int32_t sm[];
-  int32_t* sq = sm;                 // [kTile][KS] query-block pools
-  int32_t* sk = sm + kTile * KS;    // [kTile][KS] whole key-block pools (sum of the two halves)
-  const int bh = blockIdx.z, i0 = blockIdx.y * kTile, j0 = blockIdx.x * kTile;
-  const int t = threadIdx.x;
-
-  for (int idx = t; idx < kTile * C4; idx += kThreads) {
-    const int r = idx / C4, c4 = idx % C4;
-    int4 a = make_int4(0, 0, 0, 0), b = make_int4(0, 0, 0, 0);
-    if (i0 + r < nQB) a = __ldg(reinterpret_cast<const int4*>(q_pool + (size_t(bh) * nQB + i0 + r) * D) + c4);
-    if (j0 + r < nKB) {
-      const int4* p = reinterpret_cast<const int4*>(k_pool + (size_t(bh) * nKB + j0 + r) * 2 * D);
-      const int4 h0 = __ldg(p + c4), h1 = __ldg(p + C4 + c4);
-      b = make_int4(h0.x + h1.x, h0.y + h1.y, h0.z + h1.z, h0.w + h1.w);
+  constexpr int kQSteps = kSQ * C4 / kThreads, kKSteps = kSK * C4 / kThreads;
+  {
+    int4 a[kQSteps];
+#pragma unroll
+    for (int u = 0; u < kQSteps; ++u) {
+      const int idx = t + u * kThreads, r = idx / C4, c4 = idx % C4;
+      a[u] = i0 + r < nQB ? __ldg(reinterpret_cast<const int4*>(q_pool + (size_t(bh) * nQB + i0 + r) * D) + c4)
+                          : make_int4(0, 0, 0, 0);
     }
-    *reinterpret_cast<int4*>(sq + r * KS + 4 * c4) = a;
-    *reinterpret_cast<int4*>(sk + r * KS + 4 * c4) = b;
+#pragma unroll
+    for (int u = 0; u < kQSteps; ++u) {
+      const int idx = t + u * kThreads, r = idx / C4, c4 = idx % C4;
+      uint32_t hi, lo;
+      split_bytes(a[u], hi, lo);
+      const uint32_t off = swz_offset<D>(r, 4 * c4);
+      *reinterpret_cast<uint32_t*>(sm.u.t.qh + off) = hi;
+      *reinterpret_cast<uint32_t*>(sm.u.t.ql + off) = lo;
+    }
+    int4 h0[kKSteps], h1[kKSteps];
+#pragma unroll
+    for (int u = 0; u < kKSteps; ++u) {   // whole key-block pool: the sum of its two 32-row halves
+      const int idx = t + u * kThreads, r = idx / C4, c4 = idx % C4;
+      h0[u] = h1[u] = make_int4(0, 0, 0, 0);
+      if (j0 + r < nKB) {
+        const int4* p = reinterpret_cast<const int4*>(k_pool + (size_t(bh) * nKB + j0 + r) * 2 * D);
+        h0[u] = __ldg(p + c4);
+        h1[u] = __ldg(p + C4 + c4);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kKSteps; ++u) {
+      const int idx = t + u * kThreads, r = idx / C4, c4 = idx % C4;
+      uint32_t hi, lo;
+      split_bytes(make_int4(h0[u].x + h1[u].x, h0[u].y + h1[u].y, h0[u].z + h1[u].z, h0[u].w + h1[u].w), hi, lo);
+      const uint32_t off = swz_offset<D>(r, 4 * c4);
+      *reinterpret_cast<uint32_t*>(sm.u.t.kh + off) = hi;
+      *reinterpret_cast<uint32_t*>(sm.u.t.kl + off) = lo;
+    }
   }
+  fence_proxy_async_smem();   // the tensor core reads the tiles
+  tc_fence_before();
   __syncthreads();
-
-  const int tx = t & 15, ty = t >> 4;
-  long long acc[4][4];
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  if (t == 0) {
+    constexpr uint32_t kLayout = D == 128 ? 2u : 4u;   // 128B / 64B swizzle
+    constexpr uint32_t IDESC = make_idesc(2, 1, 1, false, false, kSQ, kSK);
+    const uint64_t dqh = make_sdesc(smem_u32(sm.u.t.qh), 16, 8 * D, kLayout);
+    const uint64_t dql = make_sdesc(smem_u32(sm.u.t.ql), 16, 8 * D, kLayout);
+    const uint64_t dkh = make_sdesc(smem_u32(sm.u.t.kh), 16, 8 * D, kLayout);
+    const uint64_t dkl = make_sdesc(smem_u32(sm.u.t.kl), 16, 8 * D, kLayout);
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+    for (int kk = 0; kk < D / 32; ++kk) mma_i8_ss(tmem, dqh + 2 * kk, dkh + 2 * kk, IDESC, kk > 0 ? 1u : 0u);
 #pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0;
-#pragma unroll 1
-  for (int c0 = 0; c0 < D; c0 += 16) {
-    int part[4][4];
+    for (int kk = 0; kk < D / 32; ++kk) mma_i8_ss(tmem + kSK, dqh + 2 * kk, dkl + 2 * kk, IDESC, kk > 0 ? 1u : 0u);
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int kk = 0; kk < D / 32; ++kk) mma_i8_ss(tmem + kSK, dql + 2 * kk, dkh + 2 * kk, IDESC, 1u);
 #pragma unroll
-      for (int b = 0; b < 4; ++b) part[a][b] = 0;
-#pragma unroll
-    for (int c = c0; c < c0 + 16; c += 4) {
-      int4 x[4], y[4];
-#pragma unroll
-      for (int a = 0; a < 4; ++a) x[a] = *reinterpret_cast<const int4*>(sq + (ty + 16 * a) * KS + c);
-#pragma unroll
-      for (int b = 0; b < 4; ++b) y[b] = *reinterpret_cast<const int4*>(sk + (tx + 16 * b) * KS + c);
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b)
-          part[a][b] += x[a].x * y[b].x + x[a].y * y[b].y + x[a].z * y[b].z + x[a].w * y[b].w;
-    }
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) acc[a][b] += part[a][b];
+    for (int kk = 0; kk < D / 32; ++kk)
+      mma_i8_ss(tmem + 2 * kSK, dql + 2 * kk, dkl + 2 * kk, IDESC, kk > 0 ? 1u : 0u);
+    tc_commit(&sm.done);
   }
-
+  __syncwarp();
+  // once the MMAs are done, their operand bytes are free to stage scores
+  if (mbar_wait(&sm.done, 0, &sm.abort, status, wait_limit_ns)) {
+    tc_fence_after();
+    // warp w: TMEM lanes 32 (w % 4) .. (its 32 query blocks), key-block columns 32 (w / 4) ..
+    const int r0 = 32 * (warp & 3), c0 = 32 * (warp >> 2);
+    uint32_t d1[32], d2[32], d3[32];
+    const uint32_t lane_base = uint32_t(r0) << 16;
+    tmem_ld32(tmem + lane_base + c0, d1);
+    tmem_ld32(tmem + lane_base + kSK + c0, d2);
+    tmem_ld32(tmem + lane_base + 2 * kSK + c0, d3);
+    tmem_wait_ld(d1);
+    tmem_wait_ld(d2);
+    tmem_wait_ld(d3);
+    double* stg = sm.u.stage[warp];
 #pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    const int j = j0 + tx + 16 * b;
-    if (j >= nKB) continue;
-    const double skj = (double)k_scale[size_t(bh) * nKB + j];
-    const double nj = (double)min(KB, Lk - j * KB);
+    for (int half = 0; half < 2; ++half) {
+      // the row's dots of 16 key blocks into the stage (lane = row)
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const int i = i0 + ty + 16 * a;
-      if (i < nQB) scores[(size_t(bh) * nQB + i) * nKB + j] = __ddiv_rn(__dmul_rn((double)acc[a][b], skj), nj);
+      for (int c = 0; c < 16; ++c) {
+        const int cc = 16 * half + c;
+        stg[lane * kStageLd + c] = double(16384ll * int(d1[cc]) + 128ll * int(d2[cc]) + int(d3[cc]));
+      }
+      __syncwarp();
+      // two rows per store: lanes 0-15 and 16-31 each write one row's 16 key blocks
+      const int j = j0 + c0 + 16 * half + (lane & 15);
+      if (j < nKB) {
+        const double skj = double(k_scale[size_t(bh) * nKB + j]);
+        const int nj = min(KB, Lk - j * KB);
+#pragma unroll 4
+        for (int rr = 0; rr < 32; rr += 2) {
+          const int row = rr + (lane >> 4);
+          const int i = i0 + r0 + row;
+          if (i < nQB) {
+            const double prod = __dmul_rn(stg[row * kStageLd + (lane & 15)], skj);
+            scores[(size_t(bh) * nQB + i) * nKB + j] =
+                nj == KB ? __dmul_rn(prod, 1.0 / KB) : __ddiv_rn(prod, double(nj));
+          }
+        }
+      }
+      __syncwarp();
     }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kScoreTmemCols);
   }
 }
 
@@ -311,28 +429,33 @@ __global__ void __launch_bounds__(kThreads) select_topk_kernel(const double* __r
 }  // namespace
 
 static cudaError_t launch_scores(const bsva_shape& s, const int32_t* q_pool, const int32_t* k_pool,
-                                 const float* k_scale, double* scores, cudaStream_t st) {
+                                 const float* k_scale, double* scores, uint32_t* status, cudaStream_t st) {
   const int nQB = (s.Lq + QB - 1) / QB, nKB = (s.Lk + KB - 1) / KB;
-  const size_t smem = size_t(2) * kTile * (s.d + 4) * 4;
-  dim3 g1((nKB + kTile - 1) / kTile, (nQB + kTile - 1) / kTile, s.B * s.H);
+  dim3 g1((nKB + kSK - 1) / kSK, (nQB + kSQ - 1) / kSQ, s.B * s.H);
+  // more than a third of an SM's shared memory: at most two CTAs per SM, so that their
+  // 256-column TMEM allocations always fit
+  const size_t need = (s.d == 128 ? sizeof(ScoreSmem<128>) : sizeof(ScoreSmem<64>)) + 1024;
+  const size_t smem = need > 80 * 1024 ? need : 80 * 1024;
   cudaError_t e;
   if (s.d == 128) {
     e = cudaFuncSetAttribute(score_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
-    score_kernel<128><<<g1, kThreads, smem, st>>>(q_pool, k_pool, k_scale, scores, s.Lk, nQB, nKB);
+    score_kernel<128><<<g1, kThreads, smem, st>>>(q_pool, k_pool, k_scale, scores, s.Lk, nQB, nKB, status,
+                                                  kWaitLimitNs);
   } else {
     e = cudaFuncSetAttribute(score_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
-    score_kernel<64><<<g1, kThreads, smem, st>>>(q_pool, k_pool, k_scale, scores, s.Lk, nQB, nKB);
+    score_kernel<64><<<g1, kThreads, smem, st>>>(q_pool, k_pool, k_scale, scores, s.Lk, nQB, nKB, status,
+                                                 kWaitLimitNs);
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_route_topk(const bsva_shape& s, int k_keep, const int32_t* q_pool, const int32_t* k_pool,
                               const float* k_scale, double* scores, uint8_t* kept_mask, int32_t* kept_idx,
-                              int32_t* kept_cnt, double* row_stats, cudaStream_t st) {
+                              int32_t* kept_cnt, double* row_stats, uint32_t* status, cudaStream_t st) {
   const int nQB = (s.Lq + QB - 1) / QB, nKB = (s.Lk + KB - 1) / KB;
-  cudaError_t e = launch_scores(s, q_pool, k_pool, k_scale, scores, st);
+  cudaError_t e = launch_scores(s, q_pool, k_pool, k_scale, scores, status, st);
   if (e != cudaSuccess) return e;
   dim3 g2((nQB + kThreads / 32 - 1) / (kThreads / 32), s.B * s.H);
   select_topk_kernel<<<g2, kThreads, 0, st>>>(scores, kept_mask, kept_idx, kept_cnt, row_stats, nQB, nKB, k_keep,
@@ -342,9 +465,9 @@ cudaError_t launch_route_topk(const bsva_shape& s, int k_keep, const int32_t* q_
 
 cudaError_t launch_route(const bsva_shape& s, double tau, const int32_t* q_pool, const int32_t* k_pool,
                          const float* k_scale, double* scores, uint8_t* kept_mask, int32_t* kept_idx,
-                         int32_t* kept_cnt, double* row_stats, cudaStream_t st) {
+                         int32_t* kept_cnt, double* row_stats, uint32_t* status, cudaStream_t st) {
   const int nQB = (s.Lq + QB - 1) / QB, nKB = (s.Lk + KB - 1) / KB;
-  cudaError_t e = launch_scores(s, q_pool, k_pool, k_scale, scores, st);
+  cudaError_t e = launch_scores(s, q_pool, k_pool, k_scale, scores, status, st);
   if (e != cudaSuccess) return e;
   const int neginf = std::isinf(tau) && tau < 0;
   dim3 g2((nQB + kThreads / 32 - 1) / (kThreads / 32), s.B * s.H);

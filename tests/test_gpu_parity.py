@@ -198,6 +198,48 @@ def test_masked_per_head_random_mask_with_empty_rows(gpu_lib):
     assert bool(torch.isneginf(lse[0, 1, 256:384]).all())
 
 
+def _order_edge_mask(w, rng):
+    """Per-head masks that put the attention kernel's kept-tile order at its edges. Its kept tiles
+    start at the first allowed block at or after the query block's own keys (the key block at the
+    middle of its rows, sequence ends aligned) and wrap round, so: every allowed block before
+    that anchor (the walk starts at the last one), every allowed block after it (no wrap), one far
+    block alone, everything (the ragged tail block in the middle of the walk) and a random mask."""
+    nLK = -(-w.Lk // 128)
+    m = np.zeros((w.B, w.H, w.nQB, nLK), dtype=np.uint8)
+    patterns = ["past", "future", "single", "all", "random", "past_incl"]
+    k = 0
+    for b in range(w.B):
+        for h in range(w.H):
+            pat = patterns[k % len(patterns)]
+            k += 1
+            for i in range(w.nQB):
+                kc = min(max((128 * i + 64 + w.Lk - w.Lq) // 128, 0), nLK - 1)
+                if pat == "past":
+                    m[b, h, i, :kc] = 1
+                elif pat == "past_incl":
+                    m[b, h, i, :kc + 1] = 1
+                elif pat == "future":
+                    m[b, h, i, kc + 1:] = 1
+                elif pat == "single":
+                    m[b, h, i, (kc + nLK // 2) % nLK] = 1
+                elif pat == "all":
+                    m[b, h, i, :] = 1
+                else:
+                    m[b, h, i] = rng.random(nLK) < 0.5
+    return m
+
+
+@pytest.mark.parametrize("name", ["ragged_pe", "cross", "ragged_d64"])
+def test_masked_kept_order_edges(gpu_lib, name):
+    w = workloads.get(name)
+    m = _order_edge_mask(w, np.random.default_rng(11))
+    out, lse, rep = masked_parity(gpu_lib, w, torch.from_numpy(m), softmax_scale=0.09)
+    assert_within(rep, f"kept-order edges ({name})")
+    empty = m.sum(axis=3) == 0              # e.g. the first query block of a "past" head
+    for b, h, i in zip(*np.nonzero(empty)):
+        assert bool(torch.isneginf(lse[b, h, 128 * i:min(w.Lq, 128 * i + 128)]).all())
+
+
 def test_deterministic_repeat(gpu_lib):
     w = workloads.get("ragged_pe_2x32")
     Q, K, V = inputs(w)
