@@ -13,12 +13,9 @@
 //   mu = sum s / |R|, sigma = sqrt(sum (s - mu)^2 / |R|), T = mu + tau*sigma.
 //
 // Design: two kernels.
-//  score_kernel: per head the dots are a small integer GEMM, [nQB x d] . [d x nKB]. A CTA of 256
-//   threads owns a 64 x 64 tile of (query block, key block); both pool tiles are staged in shared
-//   memory (rows padded to d+4 words: conflict-free 16-byte loads), each thread accumulates a 4 x 4
-//   block of dots (query blocks ty+16a, key blocks tx+16b) in int32 over 16 dims at a time (|q_pool|
-//   <= 16256 and |k_pool| <= 8128, so 16 products stay below 2^31) and in int64 across them, and
-//   writes the fp64 scores to the workspace, [BH, nQB, nKB].
+//  score_kernel: per head the dots are a small integer GEMM, [nQB x d] . [d x nKB], run on the
+//   tensor core as three INT8 GEMMs over the pools' signed-byte halves (details at the kernel);
+//   it writes the fp64 scores to the workspace, [BH, nQB, nKB].
 //  select_kernel: one warp per query-block row reduces mu and sigma with shuffles and compacts the
 //   kept list with ballots.
 //  select_topk_kernel: fixed-sparsity top-k over the same scores ("Ref2VA VSA", 2-stage attention
