@@ -869,13 +869,15 @@ def main():
     Qh, Kh, Vh = shard_qkv(w0, heads)
     Q, K, V = Qh.cuda(), Kh.cuda(), Vh.cuda()
 
-    measured = measure_tensor_peaks()
-    peaks = combine_peaks(_peaks(), measured)
     st = SolStep(bsva, w, args.tau, Q, K, V)
     sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
                            else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
     r, clocks = run_steps(st, args.steps, args.warmup, dist, sampler)
     bsva.check_status(st.ws)
+    # the tensor peaks after the headline: their seconds of back-to-back GEMMs would otherwise
+    # leave the GPU at its power cap during the timed steps
+    measured = measure_tensor_peaks()
+    peaks = combine_peaks(_peaks(), measured)
     work = kept_work(st.route, w)
     roof = roofline_numbers(w, work, r, peaks)
     sparsity = 1.0 - _sum_over_ranks(dist, work["kept_blocks"]) / _sum_over_ranks(dist, work["routed_blocks"])
