@@ -38,14 +38,14 @@ __all__ = [
     "quantize_q", "KVCache",
 ]
 
-ABI_VERSION = 4
+ABI_VERSION = 5
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
 
 OUT_DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA",
-          5: "DEVICE_TIMEOUT"}
+          5: "DEVICE_TIMEOUT", 6: "DEVICE_BOUNDS"}
 
 
 class BsvaError(RuntimeError):
@@ -68,12 +68,16 @@ class KVCacheStruct(ctypes.Structure):
 
 
 def lib_path() -> str:
-    return os.path.join(_HERE, "libbsva.so")
+    """The library to load: ``libbsva.so``, or the ``BSVA_DEVICE_CHECKS`` build
+    ``libbsva_checked.so`` when the environment sets ``BSVA_CHECKED=1``."""
+    name = "libbsva_checked.so" if os.environ.get("BSVA_CHECKED") == "1" else "libbsva.so"
+    return os.path.join(_HERE, name)
 
 
 _P = ctypes.c_void_p
 _SIGS = {
     "bsva_abi_version": (ctypes.c_int, []),
+    "bsva_device_checks": (ctypes.c_int, []),
     "bsva_last_error": (ctypes.c_char_p, []),
     "bsva_workspace_bytes": (ctypes.c_size_t, [Shape, ctypes.c_int]),
     "bsva_quantize_qk": (ctypes.c_int, [Shape, _P, _P, _P, _P, _P, _P, _P, _P, _P]),

@@ -642,6 +642,8 @@ int virtual_kv_residual_fwd(bsva_shape s, const int8_t* q8, const float* q_scale
                        out, lse, ws, L, st, nullptr, vtab);
 }
 
+int bsva_device_checks(void) { return kDeviceChecks ? 1 : 0; }
+
 int bsva_check_status(void* workspace, bsva_stream_t stream) {
   if (workspace == nullptr) return fail(BSVA_ERR_WORKSPACE, "workspace is NULL");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -656,6 +658,9 @@ int bsva_check_status(void* workspace, bsva_stream_t stream) {
   }
   if (word & kStatusTimeout)
     return fail(BSVA_ERR_DEVICE_TIMEOUT, "a device-side wait ran out of time; outputs of that call are invalid");
+  if (word & kStatusBounds)
+    return fail(BSVA_ERR_DEVICE_BOUNDS, "a device-side index check failed (kept count, kept list or table row out "
+                                        "of range); outputs of that call are invalid");
   return ok();
 }
 

@@ -126,7 +126,11 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int i = item % a.nQB;
   const size_t row_item = size_t(bh) * a.nQB + i;
 
-  const int n_exact = a.kept_cnt[row_item];
+  // a kept count comes from the caller's route: checked in BSVA_DEVICE_CHECKS builds
+  const int n_exact_in = a.kept_cnt[row_item];
+  const int n_exact = dcheck(n_exact_in >= 0 && n_exact_in <= a.nKB, a.status) ? n_exact_in
+                      : n_exact_in < 0                                     ? 0
+                                                                           : a.nKB;
   // Sol: the whole centroid table once some block is skipped; virtual K/V: the virtual slices' tiles
   const int n_cent = kVirt ? a.n_vtiles : (a.centroid_mode > 0 && n_exact < a.nKB) ? a.nCT : 0;
   const int N = n_exact + n_cent;
@@ -228,7 +232,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     // group metadata of centroid tile t for this lane, and the tile's first table row
     auto cent_meta = [&](int t, float& fac, float& bias, int& row) {
       if constexpr (kVirt) {   // virtual slice: 32 source groups from e.x, the first e.y of them live
-        const int2 e = a.vtab[t];
+        int2 e = a.vtab[t];
+        if (!dcheck(e.x >= 0 && e.x <= (a.nCT - 1) * 32 && e.y >= 0 && e.y <= 32, a.status)) e = make_int2(0, 0);
         const bool live = lane < e.y;
         const int G = e.x + (live ? lane : 0);   // dead lanes re-read a live entry, never past the table
         fac = sqs * cfac[G];
@@ -253,7 +258,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         if ((t & 31) == 0) {
           const int nn = t + lane;
           const int pos = nn + rot < n_exact ? nn + rot : nn + rot - n_exact;
-          chunk_j = nn < n_exact ? phys_block(a, kidx[pos]) : 0;
+          int jk = nn < n_exact ? kidx[pos] : 0;
+          if (!dcheck(jk >= 0 && jk < a.nKB, a.status)) jk = 0;   // a kept block of the caller's list
+          chunk_j = phys_block(a, jk);
           chunk_f = nn < n_exact ? sqs * a.k_scale[size_t(bh) * scale_stride + chunk_j] : 0.f;
         }
         j_next = __shfl_sync(0xffffffffu, chunk_j, t & 31);

@@ -16,6 +16,12 @@ namespace bsva {
 constexpr int QB = 128;   // query rows per block (routing granularity)
 constexpr int KB = 64;    // key rows per block
 constexpr uint32_t kStatusTimeout = 1u;   // workspace status bit: a wait ran out
+constexpr uint32_t kStatusBounds = 2u;    // workspace status bit: a device-side index check failed
+#ifdef BSVA_DEVICE_CHECKS
+constexpr bool kDeviceChecks = true;
+#else
+constexpr bool kDeviceChecks = false;
+#endif
 
 // ---------------------------------------------------------------- workspace --
 // Offsets (bytes) of the regions of the caller's workspace. All 256-aligned.
@@ -141,6 +147,18 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
       : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
+}
+
+// BSVA_DEVICE_CHECKS builds: records kStatusBounds when ok is false and returns false, so that
+// the caller clamps the value into range; other builds: true, with no code.
+__device__ __forceinline__ bool dcheck(bool ok, uint32_t* status) {
+  if constexpr (kDeviceChecks) {
+    if (!ok) {
+      if (status) atomicOr(status, kStatusBounds);
+      return false;
+    }
+  }
+  return true;
 }
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,

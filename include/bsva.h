@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define BSVA_ABI_VERSION 4
+#define BSVA_ABI_VERSION 5
 
 enum bsva_status {
   BSVA_OK = 0,
@@ -47,7 +47,9 @@ enum bsva_status {
   BSVA_ERR_UNSUPPORTED = 2,    /* device is not sm_100, d not in {64, 128}  */
   BSVA_ERR_WORKSPACE = 3,      /* workspace missing or too small            */
   BSVA_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed      */
-  BSVA_ERR_DEVICE_TIMEOUT = 5  /* a bounded device-side wait gave up        */
+  BSVA_ERR_DEVICE_TIMEOUT = 5, /* a bounded device-side wait gave up        */
+  BSVA_ERR_DEVICE_BOUNDS = 6   /* a device-side index check failed (only the
+                                  BSVA_DEVICE_CHECKS build checks)          */
 };
 
 /* Element type of the attention output `out`. */
@@ -68,6 +70,15 @@ typedef struct bsva_shape {
 /* ABI version of the loaded library; loaders compare it with BSVA_ABI_VERSION
  * ("FlashVSR Kitchen Sparse Attention", When it bites: ABI check on load). */
 int bsva_abi_version(void);
+
+/* 1 if this library was built with BSVA_DEVICE_CHECKS (libbsva_checked.so), else 0.
+ * In that build the kernels check every index they take from caller data (kept
+ * counts and kept lists of a route, table rows) before using it; a value out of
+ * range is recorded in the workspace status word (reported by bsva_check_status
+ * as BSVA_ERR_DEVICE_BOUNDS) and clamped into range, so that no access leaves its
+ * buffer; the outputs of that call are then invalid. The checks cost time; the
+ * default build does not make them. */
+int bsva_device_checks(void);
 
 /* Message for the last failed call on this thread ("" if none). The pointer
  * stays valid until the next call on the same thread. */

@@ -32,7 +32,22 @@ def test_library_builds_and_exports_every_declared_symbol():
 
 
 def test_abi_version_matches_binding():
-    assert bsva.abi_version() == bsva.ABI_VERSION == 4
+    assert bsva.abi_version() == bsva.ABI_VERSION == 5
+
+
+def test_checked_build_exports_the_same_symbols_and_says_so():
+    # the BSVA_DEVICE_CHECKS build (libbsva_checked.so) is the same ABI with index checks in the
+    # kernels; the default build reports that it makes none
+    from block_sparse_video_int8_b200 import build
+    path = build.build(checked=True)
+    lib = ctypes.CDLL(path)
+    for n in _declared():
+        assert hasattr(lib, n), n
+    lib.bsva_abi_version.restype = ctypes.c_int
+    lib.bsva_device_checks.restype = ctypes.c_int
+    assert lib.bsva_abi_version() == bsva.ABI_VERSION
+    assert lib.bsva_device_checks() == 1
+    assert bsva.load().bsva_device_checks() == 0
 
 
 def test_workspace_size_arithmetic():
